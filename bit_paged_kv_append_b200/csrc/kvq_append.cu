@@ -1,0 +1,372 @@
+// kvq_append.cu -- the fused KV-cache write: block-diagonal Hadamard rotation +
+// token-wise asymmetric INT4 quantisation + nibble packing + store into the
+// page slot, in one kernel (SAW-INT4 abstract: a fused rotation-quantisation
+// kernel integrated into paged KV-cache layouts; wispaper.ai blog section 3:
+// K~ = quant(K H_blk), V~ = quant(V H_blk), the rotation fused into the
+// KV-cache write operator with no separate kernel).
+//
+// Work unit: one (token, KV head) row of head_dim = 128 bf16 values, handled
+// entirely by one thread.  The whole 128-element transform, the min/max, the
+// quantiser and the packing then run in registers with no shuffles; the fp32
+// butterflies use sm_100's packed f32x2 add/sub/mul, pairing element i with
+// element i + 64 so every stage of stride < 64 is one packed op per pair.
+//
+// Data movement: a persistent grid (one CTA per SM); per CTA a ring of three
+// 64 KiB shared-memory stages filled by TMA tensor loads (128-byte swizzle,
+// L2 evict-first, no multicast) issued by a dedicated producer warp, which also
+// resolves each token's page slot through the page table.  Eight consumer warps
+// (256 threads = 256 rows per stage) read their row from the swizzled stage
+// without bank conflicts and write 64 B of codes + 4 B of (scale, zero) per
+// row straight to the pool.  A tile = 256 consecutive rows of the [T, H, D]
+// input = 256 / H tokens; its K rows fill one stage and its V rows the next.
+//
+// Every wait is bounded (kWaitLimitNs); out-of-range sequence ids, positions
+// and page ids are skipped and flagged in the device error word.
+#include <cudaTypedefs.h>
+
+#include "kvq_common.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr int kRows = 256;                   // (token, head) rows per stage = consumer threads
+constexpr int kThreads = kRows + 32;         // + producer warp
+constexpr int kStages = 3;
+constexpr int kHalfBytes = kRows * 128;      // one 128-byte half-row per row
+constexpr int kStageBytes = 2 * kHalfBytes;  // 64 KiB
+constexpr int kMaxTileTokens = kRows;        // H == 1
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kStages) * kStageBytes +
+                              size_t(kStages) * kMaxTileTokens * sizeof(int2) + 2 * kStages * sizeof(uint64_t);
+
+// Magic constant 1.5 * 2^23: for |v| < 2^22, the fp32 sum v + kMagic (rounded to
+// nearest even) carries rint_even(v) in its low mantissa bits.
+constexpr float kMagic = 12582912.0f;
+constexpr uint32_t kMagicBits = 0x4B400000u;
+// Sum over k = 0..7 of kMagicBits << 4k (mod 2^32): the offset the packing
+// Horner chain below accumulates from the magic bias of eight codes.
+constexpr uint32_t magic_pack_offset() {
+    uint32_t c = 0;
+    for (int k = 0; k < 8; ++k) c += kMagicBits << (4 * k);
+    return c;
+}
+constexpr uint32_t kMagicPackOffset = magic_pack_offset();
+
+struct Params {
+    CacheGeom g;
+    AppendArgs a;
+    int num_tiles;
+    int tile_tokens;  // 256 / H
+    float r_b;        // (float)(1 / sqrt((double)bdr_block))
+    int* err;
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Eight codes (as magic-biased float bits, element k in u[k]) -> one packed word,
+// element k in nibble k.
+__device__ __forceinline__ uint32_t pack8(const uint32_t (&u)[8]) {
+    uint32_t acc = u[7];
+#pragma unroll
+    for (int k = 6; k >= 0; --k) acc = (acc << 4) + u[k];
+    return acc - kMagicPackOffset;
+}
+
+// Loads this thread's row from the swizzled stage into R[i] = (x_i, x_{i+64}).
+__device__ __forceinline__ void load_row(const uint8_t* stage, int row, uint64_t (&R)[64]) {
+    const uint4* h0 = reinterpret_cast<const uint4*>(stage + row * 128);
+    const uint4* h1 = reinterpret_cast<const uint4*>(stage + kHalfBytes + row * 128);
+    const int sw = row & 7;  // 128-byte swizzle: chunk j of line L sits at chunk j ^ (L & 7)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint4 a = h0[j ^ sw];
+        const uint4 b = h1[j ^ sw];
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            R[8 * j + 2 * q] = pk(bf16_lo(aw[q]), bf16_lo(bw[q]));
+            R[8 * j + 2 * q + 1] = pk(bf16_hi(aw[q]), bf16_hi(bw[q]));
+        }
+    }
+}
+
+// Block-diagonal normalised Sylvester-Hadamard rotation of one row, fp32,
+// stages of increasing stride, then the 1/sqrt(b) multiply.
+template <int BLK>
+__device__ __forceinline__ void rotate_row(uint64_t (&R)[64], float r_b) {
+    constexpr int kPacked = BLK < 64 ? BLK : 64;  // strides below 64 stay within a packed lane
+#pragma unroll
+    for (int hs = 1; hs < kPacked; hs <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            if ((i & hs) == 0) {
+                const uint64_t a = R[i], c = R[i + hs];
+                R[i] = add2(a, c);
+                R[i + hs] = sub2(a, c);
+            }
+        }
+    }
+    if (BLK == 128) {  // stride 64 pairs the two lanes of each packed register
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            const float a = lo_of(R[i]), c = hi_of(R[i]);
+            R[i] = pk(__fadd_rn(a, c), __fsub_rn(a, c));
+        }
+    }
+    const uint64_t rr = pk(r_b, r_b);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) R[i] = mul2(R[i], rr);
+}
+
+// Token-wise asymmetric INT4 of one row: writes 64 bytes of codes and the
+// (scale, zero) word.
+__device__ __forceinline__ void quantise_store(uint64_t (&R)[64], uint8_t* codes_dst, uint32_t* sz_dst) {
+    float mn4[4], mx4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        mn4[k] = fminf(lo_of(R[k]), hi_of(R[k]));
+        mx4[k] = fmaxf(lo_of(R[k]), hi_of(R[k]));
+    }
+#pragma unroll
+    for (int i = 4; i < 64; ++i) {
+        mn4[i & 3] = min3(mn4[i & 3], lo_of(R[i]), hi_of(R[i]));
+        mx4[i & 3] = max3(mx4[i & 3], lo_of(R[i]), hi_of(R[i]));
+    }
+    float mn = min3(mn4[0], mn4[1], fminf(mn4[2], mn4[3]));
+    float mx = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+    mn = __fadd_rn(mn, 0.0f);  // -0 + +0 = +0: canonical signed zero
+    mx = __fadd_rn(mx, 0.0f);
+    const float range = __fsub_rn(mx, mn);
+    const float s32 = __fdiv_rn(range, 15.0f);
+    const __half sh = __float2half_rn(s32);
+    const __half zh = __float2half_rn(mn);
+    const float sf = __half2float(sh);
+    const float zf = __half2float(zh);
+    const float inv = sf > 0.0f ? __frcp_rn(sf) : 0.0f;
+    // The quantiser is monotone in y, so the row's extreme codes decide whether
+    // any element needs clamping; NaN fails both tests and takes the clamped path.
+    const float vmin = __fmul_rn(__fsub_rn(mn, zf), inv);
+    const float vmax = __fmul_rn(__fsub_rn(mx, zf), inv);
+    const bool in_range = (vmin >= -0.5f) && (vmax < 15.5f);
+
+    const uint64_t zz = pk(zf, zf), ii = pk(inv, inv), mm = pk(kMagic, kMagic);
+    uint32_t wa[8], wb[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        uint32_t ulo[8], uhi[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            uint64_t v = mul2(sub2(R[8 * m + k], zz), ii);
+            if (!in_range) {
+                const float a = fminf(fmaxf(lo_of(v), 0.0f), 15.0f);
+                const float b = fminf(fmaxf(hi_of(v), 0.0f), 15.0f);
+                v = pk(a, b);
+            }
+            const uint64_t u = add2(v, mm);
+            ulo[k] = __float_as_uint(lo_of(u));
+            uhi[k] = __float_as_uint(hi_of(u));
+        }
+        wa[m] = pack8(ulo);  // elements 8m .. 8m+7 -> bytes 4m .. 4m+3
+        wb[m] = pack8(uhi);  // elements 64+8m .. 64+8m+7 -> bytes 32+4m .. 32+4m+3
+    }
+    st_global_v8(codes_dst, wa);
+    st_global_v8(codes_dst + 32, wb);
+    *sz_dst = uint32_t(__half_as_ushort(sh)) | (uint32_t(__half_as_ushort(zh)) << 16);
+}
+
+template <bool ROT, int BLK>
+__device__ __forceinline__ void process_row(const uint8_t* stage, int row, float r_b, uint8_t* cdst,
+                                            uint32_t* sdst) {
+    uint64_t R[64];
+    load_row(stage, row, R);
+    if (ROT) rotate_row<BLK>(R, r_b);
+    quantise_store(R, cdst, sdst);
+}
+
+// BF16 cache: copy the row unchanged.
+__device__ __forceinline__ void copy_row(const uint8_t* stage, int row, uint8_t* dst) {
+    const uint4* h0 = reinterpret_cast<const uint4*>(stage + row * 128);
+    const uint4* h1 = reinterpret_cast<const uint4*>(stage + kHalfBytes + row * 128);
+    const int sw = row & 7;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const uint4* src = half ? h1 : h0;
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const uint4 a = src[j ^ sw], b = src[(j + 1) ^ sw];
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            st_global_v8(dst + half * 128 + j * 16, w);
+        }
+    }
+}
+
+template <int MODE, int BLK, bool ROTV>
+__global__ void __launch_bounds__(kThreads)
+    append_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = smem;
+    int2* meta = reinterpret_cast<int2*>(smem + kStages * kStageBytes);  // [stage][tile token] = (page, slot)
+    uint64_t* full = reinterpret_cast<uint64_t*>(meta + kStages * kMaxTileTokens);
+    uint64_t* empty = full + kStages;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kRows / 32);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int TT = p.tile_tokens;
+    const int H = p.g.H;
+
+    if (warp == kRows / 32) {
+        // ---------------- producer warp ----------------
+        const uint64_t pol = policy_evict_first();
+        int seqno = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+            for (int kv = 0; kv < 2; ++kv, ++seqno) {
+                const int e = seqno % kStages;
+                const uint32_t fill = seqno / kStages;
+                if (fill > 0 && !mbar_wait(&empty[e], (fill - 1) & 1)) {
+                    flag_error(p.err, kErrTimeout);
+                    return;
+                }
+                if (lane == 0) {
+                    const CUtensorMap* map = kv ? &vmap : &kmap;
+                    uint8_t* dst = stages + e * kStageBytes;
+                    mbar_expect_tx(&full[e], kStageBytes);
+                    tma_load_3d(dst, map, &full[e], 0, 0, tile * kRows, pol);
+                    tma_load_3d(dst + kHalfBytes, map, &full[e], 0, 1, tile * kRows, pol);
+                }
+                for (int tt = lane; tt < TT; tt += 32) {
+                    const int t = tile * TT + tt;
+                    int2 m = make_int2(-1, 0);
+                    if (t < p.a.num_tokens) {
+                        const int s = __ldg(p.a.tok_seq + t);
+                        const int pos = __ldg(p.a.tok_pos + t);
+                        bool ok = s >= 0 && s < p.a.num_seqs && pos >= 0 && pos / p.g.page_size < p.a.pt_stride;
+                        if (ok) {
+                            const int page = __ldg(p.a.page_table + int64_t(s) * p.a.pt_stride + pos / p.g.page_size);
+                            ok = page >= 0 && page < p.g.num_pages;
+                            if (ok) m = make_int2(page, pos % p.g.page_size);
+                        }
+                        if (!ok && kv == 0) flag_error(p.err, kErrOOB);
+                    }
+                    meta[e * kMaxTileTokens + tt] = m;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[e]);
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumer warps: thread tid owns row tid of each stage ----------------
+    const int tt = tid / H, h = tid % H;
+    int seqno = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        for (int kv = 0; kv < 2; ++kv, ++seqno) {
+            const int e = seqno % kStages;
+            const uint32_t fill = seqno / kStages;
+            if (!mbar_wait(&full[e], fill & 1)) {
+                flag_error(p.err, kErrTimeout);
+                return;
+            }
+            const int2 m = meta[e * kMaxTileTokens + tt];
+            const int t = tile * TT + tt;
+            if (t < p.a.num_tokens && m.x >= 0) {
+                const uint8_t* stage = stages + e * kStageBytes;
+                const int64_t row = (int64_t(m.x) * H + h) * p.g.page_size + m.y;
+                if (MODE == 0) {
+                    uint8_t* dst = static_cast<uint8_t*>(kv ? p.g.v_pool : p.g.k_pool) + row * 256;
+                    copy_row(stage, tid, dst);
+                } else {
+                    uint8_t* cdst = static_cast<uint8_t*>(kv ? p.g.v_pool : p.g.k_pool) + row * 64;
+                    uint32_t* sdst = (kv ? p.g.v_sz : p.g.k_sz) + row;
+                    if (kv == 0) process_row<MODE == 2, BLK>(stage, tid, p.r_b, cdst, sdst);
+                    else process_row<MODE == 2 && ROTV, BLK>(stage, tid, p.r_b, cdst, sdst);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[e]);
+        }
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// [T*H rows, 2 halves, 64 bf16] view of a [T, H, 128] bf16 input; box = one
+// 128-byte half of 256 consecutive rows, 128-byte swizzle.
+bool make_row_map(CUtensorMap* map, const void* base, int64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, 2, cuuint64_t(rows)};
+    cuuint64_t strides[2] = {128, 256};
+    cuuint32_t box[3] = {64, 1, kRows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int BLK, bool ROTV>
+cudaError_t launch_t(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
+    auto kern = append_kernel<MODE, BLK, ROTV>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    kern<<<grid, kThreads, kSmemBytes, s>>>(km, vm, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_append(const CacheGeom& g, const AppendArgs& a, int* err_word, int num_sms, cudaStream_t s) {
+    if (a.num_tokens == 0) return cudaSuccess;
+    const int64_t rows = int64_t(a.num_tokens) * g.H;
+    CUtensorMap km, vm;
+    if (!make_row_map(&km, a.k, rows) || !make_row_map(&vm, a.v, rows)) return cudaErrorInvalidValue;
+    Params p;
+    p.g = g;
+    p.a = a;
+    p.tile_tokens = kRows / g.H;
+    p.num_tiles = int((rows + kRows - 1) / kRows);
+    p.r_b = g.mode == 2 ? float(1.0 / sqrt(double(g.bdr_block))) : 1.0f;
+    p.err = err_word;
+    const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    if (g.mode == 0) return launch_t<0, 128, false>(km, vm, p, grid, s);
+    if (g.mode == 1) return launch_t<1, 128, false>(km, vm, p, grid, s);
+    switch (g.bdr_block * 2 + (g.rotate_v ? 1 : 0)) {
+        case 32: return launch_t<2, 16, false>(km, vm, p, grid, s);
+        case 33: return launch_t<2, 16, true>(km, vm, p, grid, s);
+        case 64: return launch_t<2, 32, false>(km, vm, p, grid, s);
+        case 65: return launch_t<2, 32, true>(km, vm, p, grid, s);
+        case 128: return launch_t<2, 64, false>(km, vm, p, grid, s);
+        case 129: return launch_t<2, 64, true>(km, vm, p, grid, s);
+        case 256: return launch_t<2, 128, false>(km, vm, p, grid, s);
+        case 257: return launch_t<2, 128, true>(km, vm, p, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace kvq

@@ -1,0 +1,58 @@
+// kvq_internal.h -- host-side view of libkvq.so's kernels: parameter blocks and
+// launchers shared between the C-ABI layer (kvq_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+
+struct CacheGeom {
+    int num_pages, page_size, H, Hq, D, mode, bdr_block, rotate_v;
+    void* k_pool;
+    void* v_pool;
+    uint32_t* k_sz;  // (scale, zero) fp16 pairs as one 32-bit word, scale in the low half
+    uint32_t* v_sz;
+};
+
+struct AppendArgs {
+    const void* k;
+    const void* v;
+    int num_tokens;
+    const int32_t* tok_seq;
+    const int32_t* tok_pos;
+    const int32_t* page_table;
+    int pt_stride;
+    int num_seqs;
+};
+
+struct DecodeArgs {
+    const void* q;
+    const int32_t* seq_lens;
+    const int32_t* page_table;
+    int pt_stride;
+    int batch;
+    int max_seq_len;
+    void* out;
+    int out_fp32;
+    void* workspace;
+    size_t workspace_bytes;
+};
+
+// Split-K plan for one decode call: how many splits, tokens per split.
+struct DecodePlan {
+    int num_splits;
+    int chunk;
+    size_t ws_bytes;
+};
+
+DecodePlan plan_decode(const CacheGeom& g, int batch, int max_seq_len, int num_sms);
+
+// Each returns cudaSuccess or the first launch error.
+cudaError_t launch_append(const CacheGeom& g, const AppendArgs& a, int* err_word, int num_sms, cudaStream_t s);
+cudaError_t launch_decode(const CacheGeom& g, const DecodeArgs& a, const DecodePlan& plan, int* err_word,
+                          cudaStream_t s);
+
+}  // namespace kvq

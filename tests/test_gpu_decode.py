@@ -1,0 +1,106 @@
+"""GPU parity of paged GQA decode attention (C ABI kv_decode_attn) against the float64 oracle
+over the same (oracle-verified) cache: fp32 output within ATTN_RTOL per row, bf16 output equal
+to the fp32 output rounded to nearest even."""
+import numpy as np
+import pytest
+import torch
+
+from bit_paged_kv_append_b200 import kvq, synth
+from kvq_testlib import (ATTN_RTOL, assert_pools_equal, attn_rel_err, gpu_append, gpu_decode, make_case,
+                         oracle_append, oracle_decode)
+
+pytestmark = pytest.mark.gpu
+
+WL0 = synth.WORKLOADS["single256"]
+SWEEP = [("bf16", kvq.KV_BF16, 0, False), ("int4", kvq.KV_INT4, 0, False)] + [
+    (f"bdr{b}{'kv' if rv else 'k'}", kvq.KV_INT4_BDR, b, rv) for b in (16, 32, 64, 128) for rv in (False, True)]
+
+
+def _run(c, lengths, q_seed=1, max_len=None):
+    assert gpu_append(c) == kvq.KV_OK
+    oracle_append(c)
+    assert_pools_equal(c)
+    q = synth.make_q(len(lengths), c.wl.num_q_heads, 128, seed=q_seed)
+    out32, st = gpu_decode(c, q, lengths, max_len=max_len, out_fp32=True)
+    assert st == kvq.KV_OK
+    out16, st = gpu_decode(c, q, lengths, max_len=max_len, out_fp32=False)
+    assert st == kvq.KV_OK
+    ref, skipped = oracle_decode(c, q, lengths)
+    assert skipped == 0
+    err = attn_rel_err(out32.cpu().numpy(), ref)
+    assert err <= ATTN_RTOL, err
+    assert torch.equal(out16, out32.to(torch.bfloat16))
+    return err
+
+
+@pytest.mark.parametrize("name,mode,b,rv", SWEEP, ids=[v[0] for v in SWEEP])
+def test_decode_single_sequence(name, mode, b, rv):
+    c = make_case(mode, b, rv, [256], WL0, seed=0)
+    _run(c, [256])
+
+
+@pytest.mark.parametrize("name,mode,b,rv", SWEEP, ids=[v[0] for v in SWEEP])
+def test_decode_batch16_sweep(name, mode, b, rv):
+    """16 sequences, lengths ~U[512, 4096], every variant of the block-size / K-vs-KV sweep."""
+    wl = synth.WORKLOADS["batch16"]
+    lengths = synth.seq_lengths("batch16", seed=0)
+    c = make_case(mode, b, rv, lengths, wl, seed=0)
+    _run(c, lengths)
+
+
+def test_decode_gqa8_mixed_lengths():
+    """64 query heads over 8 KV heads (G = 8), K+V rotated, lengths from 1 to a few thousand."""
+    wl = synth.WORKLOADS["mixed256"]
+    lengths = [1, 2, 15, 16, 17, 33, 500, 1024, 3001]
+    c = make_case(kvq.KV_INT4_BDR, 128, True, lengths, wl, seed=4)
+    _run(c, lengths)
+
+
+@pytest.mark.parametrize("G", [1, 2, 8])
+def test_decode_group_sizes(G):
+    wl = synth.Workload("t", 4, 4 * G, 128, 16, synth.OUTLIERS_X20, "test")
+    lengths = [70, 300]
+    c = make_case(kvq.KV_INT4_BDR, 64, False, lengths, wl, seed=G)
+    _run(c, lengths)
+
+
+def test_decode_long_sequence_many_splits():
+    """One 40k-token sequence, page size 64: split-K across the context, then the merge."""
+    wl = synth.Workload("t", 8, 32, 128, 64, synth.OUTLIERS_1PCT, "test")
+    lengths = [40_000]
+    c = make_case(kvq.KV_INT4_BDR, 128, False, lengths, wl, seed=2)
+    _run(c, lengths)
+
+
+def test_decode_empty_and_loose_bound():
+    """seq_len 0 gives a zero row; a max_seq_len bound above the real lengths changes only the plan."""
+    lengths = [0, 5, 64]
+    c = make_case(kvq.KV_INT4_BDR, 32, True, [1, 5, 64], WL0, seed=6)
+    assert gpu_append(c) == kvq.KV_OK
+    oracle_append(c)
+    q = synth.make_q(3, 32, 128, seed=3)
+    ref, _ = oracle_decode(c, q, lengths)
+    for max_len in (64, 5000):
+        out, st = gpu_decode(c, q, lengths, max_len=max_len)
+        assert st == kvq.KV_OK
+        o = out.cpu().numpy()
+        assert not o[0].any()
+        assert attn_rel_err(o, ref) <= ATTN_RTOL
+
+
+def test_decode_out_of_range_is_flagged():
+    """A length beyond the page table and a page id outside the pool are skipped and reported."""
+    c = make_case(kvq.KV_INT4, 0, False, [48], WL0, seed=8)
+    assert gpu_append(c) == kvq.KV_OK
+    oracle_append(c)
+    q = synth.make_q(1, 32, 128, seed=5)
+    pt = c.page_table.clone()
+    pt[0, 1] = -7
+    out, st = gpu_decode(c, q, [48], page_table=pt)
+    assert st == kvq.KV_ERR_OOB
+    ref, skipped = oracle_decode(c, q, [48], page_table=pt)
+    assert skipped == 16 * 32  # one page of 16 tokens, for each of the 32 query heads
+    assert attn_rel_err(out.cpu().numpy(), ref) <= ATTN_RTOL
+    big = c.page_table.shape[1] * 16 + 5
+    out, st = gpu_decode(c, q, [big], max_len=big)
+    assert st == kvq.KV_ERR_OOB
