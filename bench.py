@@ -48,10 +48,15 @@ def peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def src_hash():
+KERNEL_SOURCES = {"append_kernel": ["kvq_append.cu", "kvq_common.cuh", "kvq_internal.h"],
+                  "decode_split_kernel": ["kvq_decode.cu", "kvq_common.cuh", "kvq_internal.h"]}
+
+
+def src_hash(kernel: str):
+    """Hash of the sources one kernel is built from (the ncu counters are void once they change)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_paged_kv_append_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -62,7 +67,7 @@ def profiled_traffic(kernel: str, workload: str):
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)[kernel][workload]
-        if rec.get("src_sha") == src_hash():
+        if rec.get("src_sha") == src_hash(kernel):
             return float(rec["dram_bytes_per_launch"])
     except Exception:
         pass
