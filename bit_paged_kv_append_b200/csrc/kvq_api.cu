@@ -33,6 +33,7 @@ const char* kv_status_string(int status) {
         case KV_ERR_CUDA: return "KV_ERR_CUDA";
         case KV_ERR_OOB: return "KV_ERR_OOB";
         case KV_ERR_TIMEOUT: return "KV_ERR_TIMEOUT";
+        case KV_ERR_SCRATCH_TOO_SMALL: return "KV_ERR_SCRATCH_TOO_SMALL";
         default: return "KV_ERR_UNKNOWN";
     }
 }

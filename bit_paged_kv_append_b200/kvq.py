@@ -16,11 +16,13 @@ import torch
 from . import build as _build
 
 KV_OK, KV_ERR_INVALID, KV_ERR_UNSUPPORTED, KV_ERR_CUDA, KV_ERR_OOB, KV_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+KV_ERR_SCRATCH_TOO_SMALL = -6
+KV_NOALLOC_SCRATCH_BYTES = 8 << 20  # size of the fixed scratch behind kv_decode_attn_noalloc
 KV_BF16, KV_INT4, KV_INT4_BDR = 0, 1, 2
 HEAD_DIM = 128
 
 EXPORTS = ("kv_create_paged", "kv_append_quant", "kv_decode_workspace_bytes", "kv_decode_attn", "kv_get_error",
-           "kv_free", "kv_status_string")
+           "kv_free", "kv_status_string", "kv_decode_attn_noalloc")
 
 
 class KVQError(RuntimeError):
@@ -59,6 +61,8 @@ def load(path: str | None = None, build_if_missing: bool = True):
     lib.kv_decode_workspace_bytes.restype = Z
     lib.kv_decode_attn.argtypes = [P, P, P, P, I, I, I, P, I, P, Z, P]
     lib.kv_decode_attn.restype = I
+    lib.kv_decode_attn_noalloc.argtypes = [P, P, P, P, I, I, I, P, I, P]
+    lib.kv_decode_attn_noalloc.restype = I
     lib.kv_get_error.argtypes = [P, P]
     lib.kv_get_error.restype = I
     lib.kv_free.argtypes = [P]
@@ -119,6 +123,18 @@ def kv_decode_attn(cache, q, seq_lens, page_table, pt_stride, batch, max_seq_len
     _check(load().kv_decode_attn(cache, _ptr(q), _ptr(seq_lens), _ptr(page_table), int(pt_stride), int(batch),
                                  int(max_seq_len), _ptr(out), int(bool(out_fp32)), _ptr(workspace),
                                  int(workspace_bytes), _stream(stream)), "kv_decode_attn")
+
+
+def kv_decode_attn_noalloc(cache, q, seq_lens, page_table, pt_stride, batch, max_seq_len, out, out_fp32,
+                           stream=None):
+    """kv_decode_attn for callers that cannot allocate device memory when they decode (code inside an
+    allocator or memory pool, fixed-budget runtimes, hosts without a device allocator): the split-K scratch
+    is the library's fixed KV_NOALLOC_SCRATCH_BYTES device array, so no workspace is passed.  Calls that
+    need more scratch raise KVQError(KV_ERR_SCRATCH_TOO_SMALL); calls overlapping on the GPU share the
+    array and race, so keep them on one stream."""
+    _check(load().kv_decode_attn_noalloc(cache, _ptr(q), _ptr(seq_lens), _ptr(page_table), int(pt_stride),
+                                         int(batch), int(max_seq_len), _ptr(out), int(bool(out_fp32)),
+                                         _stream(stream)), "kv_decode_attn_noalloc")
 
 
 def kv_get_error(cache, stream=None) -> int:

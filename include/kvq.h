@@ -67,7 +67,9 @@ typedef enum {
     KV_ERR_UNSUPPORTED = -2, /* valid but not built (e.g. head_dim != 128) */
     KV_ERR_CUDA = -3,        /* a CUDA runtime call failed */
     KV_ERR_OOB = -4,         /* a kernel skipped work on an out-of-range index */
-    KV_ERR_TIMEOUT = -5      /* a kernel gave up a bounded wait (should never happen) */
+    KV_ERR_TIMEOUT = -5,     /* a kernel gave up a bounded wait (should never happen) */
+    KV_ERR_SCRATCH_TOO_SMALL = -6 /* kv_decode_attn_noalloc: the call needs more than
+                                     KV_NOALLOC_SCRATCH_BYTES of scratch; nothing launched */
 } kv_status;
 
 typedef enum {
@@ -137,6 +139,32 @@ kv_status kv_decode_attn(kv_cache* cache, const void* q, const int32_t* seq_lens
                          const int32_t* page_table, int pt_stride, int batch, int max_seq_len,
                          void* out, int out_fp32, void* workspace, size_t workspace_bytes,
                          void* stream);
+
+/* Size of the fixed device scratch array behind kv_decode_attn_noalloc. */
+#define KV_NOALLOC_SCRATCH_BYTES (8u << 20) /* 8 MiB, held on every GPU that loads the library */
+
+/* kv_decode_attn without a workspace argument, for callers that cannot allocate
+ * device memory when they decode: code running inside an allocator or memory pool
+ * that must not re-enter itself, runtimes that fix their device-memory budget up
+ * front, and plain-C hosts with no device allocator of their own.  (This entry
+ * point has no counterpart in the SAW-INT4 paper; it only changes where the
+ * split-K scratch lives.)
+ *
+ * Same arguments, kernels and results as kv_decode_attn, but the split-K scratch
+ * is a library-owned, file-scope device array of KV_NOALLOC_SCRATCH_BYTES; the
+ * call allocates nothing.  Calls whose scratch need,
+ * kv_decode_workspace_bytes(cache, batch, max_seq_len), exceeds that size return
+ * KV_ERR_SCRATCH_TOO_SMALL before launching anything.
+ *  - The first call on a device (with that device current) looks up the array's
+ *    device address with cudaGetSymbolAddress; make that first call before any
+ *    stream capture on the device.
+ *  - Every call shares the one array: calls whose kernels may overlap on the GPU
+ *    (different streams, unsynchronised threads) race on it; order them on one
+ *    stream.  No part of the array needs to start at zero: each call writes all
+ *    the scratch it later reads. */
+kv_status kv_decode_attn_noalloc(kv_cache* cache, const void* q, const int32_t* seq_lens,
+                                 const int32_t* page_table, int pt_stride, int batch, int max_seq_len,
+                                 void* out, int out_fp32, void* stream);
 
 /* Synchronise the stream, then read and clear the device error word:
  * KV_OK, KV_ERR_OOB or KV_ERR_TIMEOUT (KV_ERR_CUDA if the runtime failed). */
