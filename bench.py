@@ -49,7 +49,7 @@ def peak_hbm():
 
 
 KERNEL_SOURCES = {"append_kernel": ["kvq_append.cu", "kvq_common.cuh", "kvq_internal.h"],
-                  "decode_split_kernel": ["kvq_decode.cu", "kvq_common.cuh", "kvq_internal.h"]}
+                  "decode_mma_kernel": ["kvq_decode_mma.cu", "kvq_decode.cuh", "kvq_common.cuh", "kvq_internal.h"]}
 
 
 def src_hash(kernel: str):
@@ -374,7 +374,7 @@ def main():
     dec_gbs = dec_b / (res["decode_ms"] / 1e3) / 1e9
     dominant = "append" if res["append_ms"] >= res["decode_ms"] else "decode"
     dom_gbs = app_gbs if dominant == "append" else dec_gbs
-    traffic = profiled_traffic("append_kernel" if dominant == "append" else "decode_split_kernel", args.workload)
+    traffic = profiled_traffic("append_kernel" if dominant == "append" else "decode_mma_kernel", args.workload)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

@@ -52,7 +52,7 @@ kv_status kv_create_paged(const kv_desc* d, kv_cache** out) {
         d->bdr_block != 128)
         return KV_ERR_UNSUPPORTED;
     if (!d->k_pool || !d->v_pool || !aligned(d->k_pool, 32) || !aligned(d->v_pool, 32)) return KV_ERR_INVALID;
-    if (d->mode != KV_BF16 && (!d->k_sz || !d->v_sz || !aligned(d->k_sz, 4) || !aligned(d->v_sz, 4)))
+    if (d->mode != KV_BF16 && (!d->k_sz || !d->v_sz || !aligned(d->k_sz, 16) || !aligned(d->v_sz, 16)))
         return KV_ERR_INVALID;
     const int64_t rows = int64_t(d->num_pages) * d->num_kv_heads * d->page_size;
     if (rows > (int64_t(1) << 40)) return KV_ERR_INVALID;

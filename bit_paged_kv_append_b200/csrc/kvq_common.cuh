@@ -54,14 +54,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
         : "memory");
 }
 
+// One bounded wait: the warp is suspended (not spinning) until the phase
+// completes or kSuspendHintNs elapses; true once the phase has completed.
+constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }

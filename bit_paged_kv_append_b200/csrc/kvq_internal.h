@@ -41,10 +41,13 @@ struct DecodeArgs {
     size_t workspace_bytes;
 };
 
-// Split-K plan for one decode call: how many splits, tokens per split.
+// Split-K plan for one decode call: cached tokens per work item, the bound on
+// items per sequence and in total, and the workspace they need.
 struct DecodePlan {
-    int num_splits;
-    int chunk;
+    int item_tokens;
+    int max_splits;
+    int max_items;
+    int num_sms;
     size_t ws_bytes;
 };
 

@@ -89,7 +89,7 @@ typedef struct {
     int rotate_v;     /* KV_INT4_BDR only: 0 = rotate keys only, 1 = keys and values */
     void* k_pool;     /* device pools, layouts above; 32-byte aligned */
     void* v_pool;
-    void* k_sz;       /* device fp16x2 scale/zero arrays (INT4 modes); NULL for BF16 */
+    void* k_sz;       /* device fp16x2 scale/zero arrays (INT4 modes), 16-byte aligned; NULL for BF16 */
     void* v_sz;
 } kv_desc;
 

@@ -104,3 +104,13 @@ def test_decode_out_of_range_is_flagged():
     big = c.page_table.shape[1] * 16 + 5
     out, st = gpu_decode(c, q, [big], max_len=big)
     assert st == kvq.KV_ERR_OOB
+
+
+@pytest.mark.parametrize("ps", [1, 7, 24, 32, 48])
+def test_decode_page_sizes(ps):
+    """Page sizes that are not a multiple of 16 take the per-token gather; 32 and 48 the bulk copies."""
+    wl = synth.Workload("t", 8, 32, 128, ps, synth.OUTLIERS_X20, "test")
+    lengths = [5, 100, 333]
+    for mode, b, rv in ((kvq.KV_INT4_BDR, 128, True), (kvq.KV_INT4, 0, False), (kvq.KV_BF16, 0, False)):
+        c = make_case(mode, b, rv, lengths, wl, seed=ps)
+        _run(c, lengths)
