@@ -27,8 +27,9 @@
  *    and then multiplies by (float)(1/sqrt((double)b)).
  *  - One fp16 scale and one fp16 zero per (token, KV head) over all head_dim
  *    elements: scale = fp16(fl(max - min) / 15), zero = fp16(min);
- *    code = clamp(rint_even(fl(fl(y - zero) * fl(1 / scale))), 0, 15)
- *    (0 when scale == 0); dequantised value = code * scale + zero.
+ *    code = clamp(rint_even(fl(y - zero) * fl(1 / scale)), 0, 15), the product
+ *    rounded to an integer from its exact value (inverse 0 when scale == 0);
+ *    dequantised value = code * scale + zero.
  *  - Byte j of a row holds code 2j in its low nibble, code 2j+1 in its high one.
  *  - Query head j reads KV head j / (num_q_heads / num_kv_heads); the softmax
  *    scale is 1/sqrt(head_dim); when values are rotated, the attention output

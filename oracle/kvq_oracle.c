@@ -42,8 +42,10 @@
  *  R4 Asymmetric min/max quantiser with a float offset:
  *     scale = fp16(fl(max - min) / 15), zero = fp16(min), signed zeros of min
  *     and max canonicalised to +0 first; inv = fl(1 / float(scale)) or 0 when
- *     scale is not positive; code = clamp(rint_even(fl(fl(y - zero) * inv)),
- *     0, 15) with NaN going to 0.  Dequantised value = code * scale + zero.
+ *     scale is not positive; code = clamp(rint_even(fl(y - zero) * inv), 0, 15)
+ *     where the product fl(y - zero) * inv is taken exactly (not rounded to
+ *     fp32 before the rounding to an integer) and NaN goes to 0.  Dequantised
+ *     value = code * scale + zero.
  *  R5 Packing: byte j holds code 2j in its low nibble and code 2j+1 in its
  *     high nibble.
  *  R6 Page layout: codes uint8 [pages, H_kv, page_size, D/2]; scale/zero as
@@ -166,11 +168,13 @@ void oracle_quant_row(const float* y, int D, uint8_t* codes, uint16_t* scale_zer
         int c[2];
         for (int e = 0; e < 2; e++) {
             float t = y[2 * j + e] - zero;
-            float v = t * inv;
-            float r = rintf(v); /* default rounding mode: nearest even */
+            /* the quotient t * inv is rounded to an integer from its exact value: the
+             * product of two floats is exact in double (24 + 24 < 53 significant bits) */
+            double v = (double)t * (double)inv;
+            double r = rint(v); /* default rounding mode: nearest, ties to even */
             int code;
-            if (!(r > 0.0f)) code = 0; /* also NaN */
-            else if (r > 15.0f) code = 15;
+            if (!(r > 0.0)) code = 0; /* also NaN */
+            else if (r > 15.0) code = 15;
             else code = (int)r;
             c[e] = code;
         }

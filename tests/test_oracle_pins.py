@@ -159,11 +159,18 @@ def _golden():
     return out
 
 
-@pytest.mark.parametrize("row", ["A", "B", "C"])
+def _row_d():
+    y = np.zeros(128)
+    y[0], y[1], y[2] = -9.375, 28.125, 1.875
+    return y
+
+
+@pytest.mark.parametrize("row", ["A", "B", "C", "D"])
 def test_quant_worked_examples(row):
     g = _golden()
     i = np.arange(128)
-    y = {"A": 0.5 * (i % 16), "B": -3 + 0.25 * (i % 16), "C": np.full(128, 1.75)}[row].astype(np.float32)
+    y = {"A": 0.5 * (i % 16), "B": -3 + 0.25 * (i % 16), "C": np.full(128, 1.75), "D": _row_d()}[row].astype(
+        np.float32)
     codes, sz = oracle.quant_row(y)
     assert sz[0] == int(g[f"{row}.scale"][0], 16)
     assert sz[1] == int(g[f"{row}.zero"][0], 16)
@@ -200,6 +207,25 @@ def test_quant_error_bound_and_monotone(mag):
         assert np.max(np.abs(xh - y)) <= bound
         order = np.argsort(y, kind="stable")
         assert np.all(np.diff(c[order].astype(int)) >= 0)
+
+
+def test_quant_rounds_the_exact_quotient():
+    """The code is the integer nearest the exact product fl(y - zero) * fl(1/scale) (ties to
+    even), checked with rational arithmetic on random rows."""
+    from fractions import Fraction
+
+    rng = np.random.default_rng(17)
+    for _ in range(50):
+        y = (rng.standard_normal(128) * rng.choice([0.01, 1.0, 40.0])).astype(np.float32)
+        codes, sz = oracle.quant_row(y)
+        c = oracle.unpack_codes(codes)
+        scale = np.uint16(sz[0]).view(np.float16).astype(np.float32)
+        zero = np.uint16(sz[1]).view(np.float16).astype(np.float32)
+        inv = np.float32(1) / scale if scale > 0 else np.float32(0)
+        for e in range(128):
+            q = Fraction(float(np.float32(y[e]) - zero)) * Fraction(float(inv))
+            r = round(q)  # Fraction rounding: nearest, ties to even
+            assert c[e] == (0 if r <= 0 else min(15, r))
 
 
 def test_quant_signed_zero_row_is_canonical():
