@@ -44,7 +44,7 @@ kv_status kv_create_paged(const kv_desc* d, kv_cache** out) {
     if (d->num_pages < 1 || d->page_size < 1 || d->page_size > 1024) return KV_ERR_INVALID;
     if (d->num_kv_heads < 1 || d->num_q_heads < 1 || d->num_q_heads % d->num_kv_heads) return KV_ERR_INVALID;
     if (d->head_dim != kvq::kHeadDim) return KV_ERR_UNSUPPORTED;
-    if (128 % d->num_kv_heads) return KV_ERR_UNSUPPORTED;
+    if (32 % d->num_kv_heads) return KV_ERR_UNSUPPORTED;
     const int G = d->num_q_heads / d->num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return KV_ERR_UNSUPPORTED;
     if (d->mode < KV_BF16 || d->mode > KV_INT4_BDR) return KV_ERR_INVALID;

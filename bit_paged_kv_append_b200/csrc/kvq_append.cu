@@ -8,17 +8,24 @@
 // Work unit: one (token, KV head) row of head_dim = 128 bf16 values, handled
 // entirely by one thread.  The whole 128-element transform, the min/max, the
 // quantiser and the packing then run in registers with no shuffles; the fp32
-// butterflies use sm_100's packed f32x2 add/sub/mul, pairing element i with
-// element i + 64 so every stage of stride < 64 is one packed op per pair.
+// butterflies use sm_100's packed f32x2 adds, pairing element i with element
+// i + 64 so every stage of stride < 64 is one packed op per pair.  The compiler
+// contracts a packed multiply followed by a packed add into one fused op even
+// when both carry an explicit rounding mode, so the only packed multiply used
+// is a deliberate fma, and the 1/sqrt(b) normalisation is scalar.
 //
 // Data movement: a persistent grid (one CTA per SM); per CTA a ring of three
-// 64 KiB shared-memory stages filled by TMA tensor loads (128-byte swizzle,
-// L2 evict-first, no multicast) issued by a dedicated producer warp, which also
-// resolves each token's page slot through the page table.  Eight consumer warps
-// (256 threads = 256 rows per stage) read their row from the swizzled stage
-// without bank conflicts and write 64 B of codes + 4 B of (scale, zero) per
-// row straight to the pool.  A tile = 256 consecutive rows of the [T, H, D]
-// input = 256 / H tokens; its K rows fill one stage and its V rows the next.
+// 56 KiB shared-memory stages filled by TMA tensor loads (128-byte swizzle,
+// L2 evict-first, no multicast) issued by a producer warp, which also resolves
+// each token's page slot (ids loaded one tile ahead, page lookups overlapped
+// with the tile's copies, a 2-slot meta ring).  Seven consumer warps (224
+// threads = 224 rows per stage; with the producer, two warps per SM
+// sub-partition, so a thread may hold ~200 registers) read their row from the
+// swizzled stage without bank conflicts, write 64 B of codes + 4 B of (scale,
+// zero) per row straight to the pool, and free the stage on an mbarrier: no
+// block-wide barrier in the loop.  A tile = 224 consecutive rows of the
+// [T, H, D] input = 224 / H tokens (H divides 32); its K rows fill one stage and
+// its V rows the next.
 //
 // Every wait is bounded (kWaitLimitNs); out-of-range sequence ids, positions
 // and page ids are skipped and flagged in the device error word.
@@ -30,14 +37,14 @@
 namespace kvq {
 namespace {
 
-constexpr int kRows = 256;                   // (token, head) rows per stage = consumer threads
-constexpr int kThreads = kRows + 32;         // + producer warp
+constexpr int kRows = 224;                   // (token, head) rows per stage = consumer threads (7 warps)
+constexpr int kThreads = kRows + 32;         // + one producer warp: 8 warps, two per SM sub-partition
 constexpr int kStages = 3;
 constexpr int kHalfBytes = kRows * 128;      // one 128-byte half-row per row
-constexpr int kStageBytes = 2 * kHalfBytes;  // 64 KiB
+constexpr int kStageBytes = 2 * kHalfBytes;  // 56 KiB (a multiple of 1 KiB: swizzle atoms stay aligned)
 constexpr int kMaxTileTokens = kRows;        // H == 1
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kStages) * kStageBytes +
-                              size_t(kStages) * kMaxTileTokens * sizeof(int2) + 2 * kStages * sizeof(uint64_t);
+                              2 * size_t(kMaxTileTokens) * sizeof(int2) + 2 * kStages * sizeof(uint64_t);
 
 // Magic constant 1.5 * 2^23: for |v| < 2^22, the fp32 sum v + kMagic (rounded to
 // nearest even) carries rint_even(v) in its low mantissa bits.
@@ -56,7 +63,7 @@ struct Params {
     CacheGeom g;
     AppendArgs a;
     int num_tiles;
-    int tile_tokens;  // 256 / H
+    int tile_tokens;  // kRows / H
     float r_b;        // (float)(1 / sqrt((double)bdr_block))
     int* err;
 };
@@ -74,7 +81,7 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&u)[8]) {
 }
 
 // Loads this thread's row from the swizzled stage into R[i] = (x_i, x_{i+64}).
-__device__ __forceinline__ void load_row(const uint8_t* stage, int row, uint64_t (&R)[64]) {
+__device__ __forceinline__ void load_row(const uint8_t* stage, int row, float2 (&R)[64]) {
     const uint4* h0 = reinterpret_cast<const uint4*>(stage + row * 128);
     const uint4* h1 = reinterpret_cast<const uint4*>(stage + kHalfBytes + row * 128);
     const int sw = row & 7;  // 128-byte swizzle: chunk j of line L sits at chunk j ^ (L & 7)
@@ -86,53 +93,77 @@ __device__ __forceinline__ void load_row(const uint8_t* stage, int row, uint64_t
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            R[8 * j + 2 * q] = pk(bf16_lo(aw[q]), bf16_lo(bw[q]));
-            R[8 * j + 2 * q + 1] = pk(bf16_hi(aw[q]), bf16_hi(bw[q]));
+            R[8 * j + 2 * q] = make_float2(bf16_lo(aw[q]), bf16_lo(bw[q]));
+            R[8 * j + 2 * q + 1] = make_float2(bf16_hi(aw[q]), bf16_hi(bw[q]));
         }
     }
 }
 
 // Block-diagonal normalised Sylvester-Hadamard rotation of one row, fp32,
-// stages of increasing stride, then the 1/sqrt(b) multiply.
+// stages of increasing stride, then the 1/sqrt(b) multiply.  The butterflies
+// are packed adds (no multiply anywhere to contract with); the normalisation
+// uses scalar multiplies that are never merged into a later add.
 template <int BLK>
-__device__ __forceinline__ void rotate_row(uint64_t (&R)[64], float r_b) {
+__device__ __forceinline__ void rotate_row(float2 (&R)[64], float r_b) {
     constexpr int kPacked = BLK < 64 ? BLK : 64;  // strides below 64 stay within a packed lane
 #pragma unroll
     for (int hs = 1; hs < kPacked; hs <<= 1) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
             if ((i & hs) == 0) {
-                const uint64_t a = R[i], c = R[i + hs];
-                R[i] = add2(a, c);
-                R[i + hs] = sub2(a, c);
+                const float2 a = R[i], c = R[i + hs];
+                R[i] = __fadd2_rn(a, c);
+                R[i + hs] = __fadd2_rn(a, make_float2(-c.x, -c.y));  // a - c, exactly
             }
         }
     }
     if (BLK == 128) {  // stride 64 pairs the two lanes of each packed register
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const float a = lo_of(R[i]), c = hi_of(R[i]);
-            R[i] = pk(__fadd_rn(a, c), __fsub_rn(a, c));
-        }
+        for (int i = 0; i < 64; ++i) R[i] = make_float2(__fadd_rn(R[i].x, R[i].y), __fsub_rn(R[i].x, R[i].y));
     }
-    const uint64_t rr = pk(r_b, r_b);
 #pragma unroll
-    for (int i = 0; i < 64; ++i) R[i] = mul2(R[i], rr);
+    for (int i = 0; i < 64; ++i) R[i] = make_float2(__fmul_rn(R[i].x, r_b), __fmul_rn(R[i].y, r_b));
+}
+
+// Codes of a row into 16 packed words: wa = elements 0..63, wb = elements 64..127.
+// u = fma(y - zero, inv, 1.5 * 2^23) rounds the exact quotient to the nearest
+// integer (ties to even) in its low mantissa bits.  CLAMP maps quotients below 0
+// (or NaN) to 0 and above 15 to 15; rows whose extreme codes are in range skip it.
+template <bool CLAMP>
+__device__ __forceinline__ void quantise_pack(const float2 (&R)[64], float zf, float inv, uint32_t (&wa)[8],
+                                              uint32_t (&wb)[8]) {
+    const float2 nz = make_float2(-zf, -zf), ii = make_float2(inv, inv), mm = make_float2(kMagic, kMagic);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        uint32_t ulo[8], uhi[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            float2 u = __ffma2_rn(__fadd2_rn(R[8 * m + k], nz), ii, mm);
+            if (CLAMP) {
+                u.x = u.x > kMagic ? fminf(u.x, kMagic + 15.0f) : kMagic;
+                u.y = u.y > kMagic ? fminf(u.y, kMagic + 15.0f) : kMagic;
+            }
+            ulo[k] = __float_as_uint(u.x);
+            uhi[k] = __float_as_uint(u.y);
+        }
+        wa[m] = pack8(ulo);  // elements 8m .. 8m+7 -> bytes 4m .. 4m+3
+        wb[m] = pack8(uhi);  // elements 64+8m .. 64+8m+7 -> bytes 32+4m .. 32+4m+3
+    }
 }
 
 // Token-wise asymmetric INT4 of one row: writes 64 bytes of codes and the
 // (scale, zero) word.
-__device__ __forceinline__ void quantise_store(uint64_t (&R)[64], uint8_t* codes_dst, uint32_t* sz_dst) {
+__device__ __forceinline__ void quantise_store(const float2 (&R)[64], uint8_t* codes_dst, uint32_t* sz_dst) {
     float mn4[4], mx4[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        mn4[k] = fminf(lo_of(R[k]), hi_of(R[k]));
-        mx4[k] = fmaxf(lo_of(R[k]), hi_of(R[k]));
+        mn4[k] = fminf(R[k].x, R[k].y);
+        mx4[k] = fmaxf(R[k].x, R[k].y);
     }
 #pragma unroll
     for (int i = 4; i < 64; ++i) {
-        mn4[i & 3] = min3(mn4[i & 3], lo_of(R[i]), hi_of(R[i]));
-        mx4[i & 3] = max3(mx4[i & 3], lo_of(R[i]), hi_of(R[i]));
+        mn4[i & 3] = min3(mn4[i & 3], R[i].x, R[i].y);
+        mx4[i & 3] = max3(mx4[i & 3], R[i].x, R[i].y);
     }
     float mn = min3(mn4[0], mn4[1], fminf(mn4[2], mn4[3]));
     float mx = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
@@ -145,32 +176,16 @@ __device__ __forceinline__ void quantise_store(uint64_t (&R)[64], uint8_t* codes
     const float sf = __half2float(sh);
     const float zf = __half2float(zh);
     const float inv = sf > 0.0f ? __frcp_rn(sf) : 0.0f;
-    // The quantiser is monotone in y, so the row's extreme codes decide whether
-    // any element needs clamping; NaN fails both tests and takes the clamped path.
-    const float vmin = __fmul_rn(__fsub_rn(mn, zf), inv);
-    const float vmax = __fmul_rn(__fsub_rn(mx, zf), inv);
-    const bool in_range = (vmin >= -0.5f) && (vmax < 15.5f);
-
-    const uint64_t zz = pk(zf, zf), ii = pk(inv, inv), mm = pk(kMagic, kMagic);
+    // The quantiser is monotone in y, so the row's extreme codes decide whether any
+    // element needs clamping; NaN fails both tests and takes the clamped path.
+    const float umin = __fmaf_rn(__fsub_rn(mn, zf), inv, kMagic);
+    const float umax = __fmaf_rn(__fsub_rn(mx, zf), inv, kMagic);
+    const bool in_range = (umin >= kMagic) && (umax <= kMagic + 15.0f);
     uint32_t wa[8], wb[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        uint32_t ulo[8], uhi[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            uint64_t v = mul2(sub2(R[8 * m + k], zz), ii);
-            if (!in_range) {
-                const float a = fminf(fmaxf(lo_of(v), 0.0f), 15.0f);
-                const float b = fminf(fmaxf(hi_of(v), 0.0f), 15.0f);
-                v = pk(a, b);
-            }
-            const uint64_t u = add2(v, mm);
-            ulo[k] = __float_as_uint(lo_of(u));
-            uhi[k] = __float_as_uint(hi_of(u));
-        }
-        wa[m] = pack8(ulo);  // elements 8m .. 8m+7 -> bytes 4m .. 4m+3
-        wb[m] = pack8(uhi);  // elements 64+8m .. 64+8m+7 -> bytes 32+4m .. 32+4m+3
-    }
+    if (in_range)
+        quantise_pack<false>(R, zf, inv, wa, wb);
+    else
+        quantise_pack<true>(R, zf, inv, wa, wb);
     st_global_v8(codes_dst, wa);
     st_global_v8(codes_dst + 32, wb);
     *sz_dst = uint32_t(__half_as_ushort(sh)) | (uint32_t(__half_as_ushort(zh)) << 16);
@@ -179,7 +194,7 @@ __device__ __forceinline__ void quantise_store(uint64_t (&R)[64], uint8_t* codes
 template <bool ROT, int BLK>
 __device__ __forceinline__ void process_row(const uint8_t* stage, int row, float r_b, uint8_t* cdst,
                                             uint32_t* sdst) {
-    uint64_t R[64];
+    float2 R[64];
     load_row(stage, row, R);
     if (ROT) rotate_row<BLK>(R, r_b);
     quantise_store(R, cdst, sdst);
@@ -203,37 +218,56 @@ __device__ __forceinline__ void copy_row(const uint8_t* stage, int row, uint8_t*
 }
 
 template <int MODE, int BLK, bool ROTV>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
     append_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
-    int2* meta = reinterpret_cast<int2*>(smem + kStages * kStageBytes);  // [stage][tile token] = (page, slot)
-    uint64_t* full = reinterpret_cast<uint64_t*>(meta + kStages * kMaxTileTokens);
+    int2* meta = reinterpret_cast<int2*>(smem + kStages * kStageBytes);  // [tile parity][tile token] = (page, slot)
+    uint64_t* full = reinterpret_cast<uint64_t*>(meta + 2 * kMaxTileTokens);
     uint64_t* empty = full + kStages;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    const int TT = p.tile_tokens;
+    const int H = p.g.H;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kRows / 32);
+        for (int e = 0; e < kStages; ++e) {
+            mbar_init(&full[e], 1);
+            mbar_init(&empty[e], kRows / 32);
         }
         fence_mbar_init();
     }
     __syncthreads();
 
-    const int TT = p.tile_tokens;
-    const int H = p.g.H;
-
     if (warp == kRows / 32) {
         // ---------------- producer warp ----------------
+        // Per tile: load the next tile's (sequence, position) ids, issue this tile's K and V
+        // stage copies, resolve this tile's page slots (one dependent load, overlapped with
+        // the copies) into its meta slot, then release both stages.
         const uint64_t pol = policy_evict_first();
-        int seqno = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        constexpr int kPerLane = (kMaxTileTokens + 31) / 32;
+        int sq[kPerLane], po[kPerLane];
+        auto load_ids = [&](int tile, int (&a)[kPerLane], int (&b)[kPerLane]) {
+#pragma unroll
+            for (int r = 0; r < kPerLane; ++r) {
+                const int tt = lane + 32 * r;
+                const int t = tile * TT + tt;
+                const bool in = tile < p.num_tiles && tt < TT && t < p.a.num_tokens;
+                a[r] = in ? __ldg(p.a.tok_seq + t) : -1;
+                b[r] = in ? __ldg(p.a.tok_pos + t) : -1;
+            }
+        };
+        load_ids(blockIdx.x, sq, po);
+        int seqno = 0, n = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++n) {
+            int nsq[kPerLane], npo[kPerLane];
+            load_ids(tile + gridDim.x, nsq, npo);
+            int es[2];
             for (int kv = 0; kv < 2; ++kv, ++seqno) {
                 const int e = seqno % kStages;
                 const uint32_t fill = seqno / kStages;
+                es[kv] = e;
                 if (fill > 0 && !mbar_wait(&empty[e], (fill - 1) & 1)) {
                     flag_error(p.err, kErrTimeout);
                     return;
@@ -245,24 +279,37 @@ __global__ void __launch_bounds__(kThreads)
                     tma_load_3d(dst, map, &full[e], 0, 0, tile * kRows, pol);
                     tma_load_3d(dst + kHalfBytes, map, &full[e], 0, 1, tile * kRows, pol);
                 }
-                for (int tt = lane; tt < TT; tt += 32) {
+            }
+            // the meta slot of tile n was last read for tile n - 2, whose stages the waits above freed
+            int2* mt = meta + (n & 1) * kMaxTileTokens;
+#pragma unroll
+            for (int r = 0; r < kPerLane; ++r) {
+                const int tt = lane + 32 * r;
+                if (tt < TT) {
                     const int t = tile * TT + tt;
                     int2 m = make_int2(-1, 0);
                     if (t < p.a.num_tokens) {
-                        const int s = __ldg(p.a.tok_seq + t);
-                        const int pos = __ldg(p.a.tok_pos + t);
-                        bool ok = s >= 0 && s < p.a.num_seqs && pos >= 0 && pos / p.g.page_size < p.a.pt_stride;
+                        const int sid = sq[r], pos = po[r];
+                        bool ok = sid >= 0 && sid < p.a.num_seqs && pos >= 0 && pos / p.g.page_size < p.a.pt_stride;
                         if (ok) {
-                            const int page = __ldg(p.a.page_table + int64_t(s) * p.a.pt_stride + pos / p.g.page_size);
+                            const int page = __ldg(p.a.page_table + int64_t(sid) * p.a.pt_stride + pos / p.g.page_size);
                             ok = page >= 0 && page < p.g.num_pages;
                             if (ok) m = make_int2(page, pos % p.g.page_size);
                         }
-                        if (!ok && kv == 0) flag_error(p.err, kErrOOB);
+                        if (!ok) flag_error(p.err, kErrOOB);
                     }
-                    meta[e * kMaxTileTokens + tt] = m;
+                    mt[tt] = m;
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full[e]);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&full[es[0]]);
+                mbar_arrive(&full[es[1]]);
+            }
+#pragma unroll
+            for (int r = 0; r < kPerLane; ++r) {
+                sq[r] = nsq[r];
+                po[r] = npo[r];
             }
         }
         return;
@@ -270,8 +317,9 @@ __global__ void __launch_bounds__(kThreads)
 
     // ---------------- consumer warps: thread tid owns row tid of each stage ----------------
     const int tt = tid / H, h = tid % H;
-    int seqno = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    int seqno = 0, n = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++n) {
+        int2 m = make_int2(-1, 0);
         for (int kv = 0; kv < 2; ++kv, ++seqno) {
             const int e = seqno % kStages;
             const uint32_t fill = seqno / kStages;
@@ -279,7 +327,7 @@ __global__ void __launch_bounds__(kThreads)
                 flag_error(p.err, kErrTimeout);
                 return;
             }
-            const int2 m = meta[e * kMaxTileTokens + tt];
+            if (kv == 0) m = meta[(n & 1) * kMaxTileTokens + tt];
             const int t = tile * TT + tt;
             if (t < p.a.num_tokens && m.x >= 0) {
                 const uint8_t* stage = stages + e * kStageBytes;
@@ -313,7 +361,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [T*H rows, 2 halves, 64 bf16] view of a [T, H, 128] bf16 input; box = one
-// 128-byte half of 256 consecutive rows, 128-byte swizzle.
+// 128-byte half of kRows consecutive rows, 128-byte swizzle.
 bool make_row_map(CUtensorMap* map, const void* base, int64_t rows) {
     auto fn = encode_fn();
     if (!fn) return false;

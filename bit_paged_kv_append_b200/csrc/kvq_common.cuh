@@ -1,6 +1,6 @@
 // kvq_common.cuh -- device helpers shared by the append and decode kernels of
-// libkvq.so (sm_100a only): bounded mbarrier waits, TMA tensor loads, packed
-// fp32x2 arithmetic and the device error word.
+// libkvq.so (sm_100a only): bounded mbarrier waits, TMA tensor loads, 3-input
+// min/max and the device error word.
 #pragma once
 
 #include <cuda.h>
@@ -82,6 +82,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 
 // ---- TMA (no multicast anywhere in this library) ----------------------------
 
+// Orders this thread's earlier generic-proxy accesses of shared memory before
+// later async-proxy (TMA / bulk copy) accesses of it.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
                                             int c2, uint64_t policy) {
     asm volatile(
@@ -97,38 +101,7 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
-// ---- packed fp32x2 arithmetic (sm_100a), each lane one IEEE RN operation ----
-
-__device__ __forceinline__ uint64_t pk(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ float lo_of(uint64_t v) {
-    float lo;
-    asm("mov.b64 {%0, _}, %1;" : "=f"(lo) : "l"(v));
-    return lo;
-}
-__device__ __forceinline__ float hi_of(uint64_t v) {
-    float hi;
-    asm("mov.b64 {_, %0}, %1;" : "=f"(hi) : "l"(v));
-    return hi;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
+// ---- 3-input min / max (sm_100a) ----------------------------------------------
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;

@@ -198,52 +198,53 @@ __global__ void __launch_bounds__(kThreads) bf16_split_kernel(Params p) {
 
 // ---------------------------------------------------------------- merge --------
 
-// One CTA per (sequence, query head): merge the sequence's splits (their
-// statistics fetched in parallel, 128 splits at a time), normalise, rotate back
+// One CTA per (sequence, query head): merge the sequence's splits (statistics
+// fetched once, 128 splits at a time, partial outputs loaded 8 at a time),
+// normalise, rotate back
 // when values were rotated (o H_blk; H_blk is its own inverse), store bf16 (round
 // to nearest even of the fp32 value) or fp32.  An empty sequence gives zeros.
 __global__ void __launch_bounds__(kThreads) merge_kernel(Params p, int rotate_out) {
     __shared__ float wts[kThreads];
-    __shared__ float red[kWarps];
+    __shared__ float red[2][kWarps];
     __shared__ float buf[kHeadDim];
     const int row = blockIdx.x;  // s * Hq + j
     const int Hq = p.g.Hq;
     const int s = row / Hq, j = row % Hq;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = (decode_len(p, s) + p.item_tokens - 1) / p.item_tokens;
-    // global max of the split maxima
-    float M = -INFINITY;
-    for (int k = tid; k < n; k += kThreads) M = fmaxf(M, p.ws_ml[partial_row(p, s, k, j)].x);
-    M = warp_max(M);
-    if (lane == 0) red[warp] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
-    float acc = 0.0f, lpart = 0.0f;
+    const int64_t stride = int64_t(Hq) * kHeadDim;  // next split, same query head
+    float acc = 0.0f, l = 0.0f, M = -INFINITY;
+    // splits in tiles of 128: thread t fetches the statistics of split k0 + t, the tile's
+    // weights go through shared memory, every thread then sums its dimension over the tile
     for (int k0 = 0; k0 < n; k0 += kThreads) {
         const int cnt = min(kThreads, n - k0);
-        if (tid < cnt) {
-            const float2 ml = p.ws_ml[partial_row(p, s, k0 + tid, j)];
-            const float f = (ml.x == -INFINITY) ? 0.0f : fast_exp2(ml.x - M);
-            wts[tid] = f;
-            lpart += f * ml.y;
-        }
+        const float2 ml = tid < cnt ? p.ws_ml[partial_row(p, s, k0 + tid, j)] : make_float2(-INFINITY, 0.0f);
+        float tm = warp_max(ml.x);
+        if (lane == 0) red[0][warp] = tm;
         __syncthreads();
+        tm = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
+        const float Mn = fmaxf(M, tm);
+        const float f = (ml.x == -INFINITY) ? 0.0f : fast_exp2(ml.x - Mn);
+        wts[tid] = f;
+        const float lt = warp_sum(f * ml.y);
+        if (lane == 0) red[1][warp] = lt;
+        __syncthreads();
+        const float rescale = (M == -INFINITY) ? 0.0f : fast_exp2(M - Mn);
+        l = l * rescale + (red[1][0] + red[1][1] + red[1][2] + red[1][3]);
+        acc *= rescale;
+        M = Mn;
         const float* src = p.ws_o + partial_row(p, s, k0, j) * kHeadDim + tid;
-        const int64_t stride = int64_t(Hq) * kHeadDim;  // next split, same query head
         int t = 0;
-        for (; t + 4 <= cnt; t += 4) {
-            const float o0 = src[(t + 0) * stride], o1 = src[(t + 1) * stride];
-            const float o2 = src[(t + 2) * stride], o3 = src[(t + 3) * stride];
-            acc += wts[t] * o0 + wts[t + 1] * o1 + wts[t + 2] * o2 + wts[t + 3] * o3;
+        for (; t + 8 <= cnt; t += 8) {
+            float o[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) o[u] = src[(t + u) * stride];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc += wts[t + u] * o[u];
         }
         for (; t < cnt; ++t) acc += wts[t] * src[t * stride];
         __syncthreads();
     }
-    const float lw = warp_sum(lpart);
-    if (lane == 0) red[warp] = lw;
-    __syncthreads();
-    const float l = red[0] + red[1] + red[2] + red[3];
     float res = l > 0.0f ? acc / l : 0.0f;
     if (rotate_out) {
         buf[tid] = res;

@@ -82,7 +82,7 @@ typedef enum {
 typedef struct {
     int num_pages;    /* pages in each pool */
     int page_size;    /* tokens per page, 1..1024 */
-    int num_kv_heads; /* H_kv, must divide 128 */
+    int num_kv_heads; /* H_kv: 1, 2, 4, 8, 16 or 32 */
     int num_q_heads;  /* H_q = G * H_kv with G in {1, 2, 4, 8} */
     int head_dim;     /* must be 128 */
     int mode;         /* kv_mode */

@@ -55,6 +55,7 @@ def _desc(**kw):
     (dict(num_q_heads=30), kvq.KV_ERR_INVALID),
     (dict(head_dim=64), kvq.KV_ERR_UNSUPPORTED),
     (dict(num_kv_heads=3, num_q_heads=12), kvq.KV_ERR_UNSUPPORTED),
+    (dict(num_kv_heads=64, num_q_heads=64), kvq.KV_ERR_UNSUPPORTED),
     (dict(num_q_heads=8 * 16), kvq.KV_ERR_UNSUPPORTED),
     (dict(mode=7), kvq.KV_ERR_INVALID),
     (dict(bdr_block=8), kvq.KV_ERR_UNSUPPORTED),
