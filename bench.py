@@ -1,22 +1,32 @@
 #!/usr/bin/env python
 """Benchmark of the SAW-INT4 KV-cache write/read hot path on B200.
 
-One step = one pass of the whole path over one batch: the fused BDR + INT4 append
-of every token of the batch into the paged cache (one kv_append_quant launch),
-then one paged GQA decode step per sequence (kv_decode_attn: split + merge
-kernels).  Default workload: 16 sequences with lengths ~U[512, 4096] (seed 0),
-8 KV heads, 32 query heads, head_dim 128, page size 16, shuffled page table,
-K/V ~ N(0,1) with 4 outlier channels per head x20, BDR block 128 on keys.
+One step = one pass of the whole path over one batch of a serving workload:
+the fused BDR + INT4 appends of the step's new tokens into the paged cache
+(kv_append_quant), then one paged GQA decode step (kv_decode_attn: split +
+merge kernels).  Workloads (synthetic, seeded; K/V ~ N(0,1) with outlier
+channels, q ~ N(0,1)):
 
-Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on the
-host cores instead, on a bounded sample of the same workload.
+  batch16      (default) 16 sequences, lengths ~U[512, 4096], page size 16: a step
+               appends every token of every sequence, then decodes all 16.
+  decode64x8k  64 x 8192 cached tokens (prefilled, untimed): a step appends 1
+               token per sequence at position 8192 and decodes 8193 tokens each.
+  mixed256     256 sequences, lengths log-uniform [1024, 32768], 64 query heads,
+               K and V rotated (prefilled, untimed): a step appends a 2048-token
+               chunk to 8 sequences and 1 token to each of the other 248, then
+               decodes those 248.
+  long1m       1 sequence x 1,048,576 tokens, page size 64: a step appends the
+               context in 128 chunks of 8192 tokens, then decodes it (split-K).
+Steps rewrite the same slots each time, so every step does the same work.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+the host cores instead, on a bounded sample of the same workload.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
-import math
 import os
 import subprocess
 import sys
@@ -37,7 +47,14 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 VARIANTS = [("bf16", kvq.KV_BF16, 0, False), ("int4", kvq.KV_INT4, 0, False)] + [
     (f"bdr{b}_{'kv' if rv else 'k'}", kvq.KV_INT4_BDR, b, rv) for b in (16, 32, 64, 128) for rv in (False, True)]
-HEADLINE = "bdr128_k"
+# the variant each workload is quoted on (the blog's section 4: block 128, keys only; K and V for mixed serving)
+HEADLINE = {"batch16": ("bdr128_k", kvq.KV_INT4_BDR, 128, False),
+            "single256": ("bdr128_k", kvq.KV_INT4_BDR, 128, False),
+            "decode64x8k": ("bdr128_k", kvq.KV_INT4_BDR, 128, False),
+            "mixed256": ("bdr128_kv", kvq.KV_INT4_BDR, 128, True),
+            "long1m": ("bdr128_k", kvq.KV_INT4_BDR, 128, False)}
+KERNEL_SOURCES = {"append_kernel": ["kvq_append.cu", "kvq_common.cuh", "kvq_internal.h"],
+                  "decode_mma_kernel": ["kvq_decode_mma.cu", "kvq_decode.cuh", "kvq_common.cuh", "kvq_internal.h"]}
 
 
 def peak_hbm():
@@ -46,10 +63,6 @@ def peak_hbm():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
-
-
-KERNEL_SOURCES = {"append_kernel": ["kvq_append.cu", "kvq_common.cuh", "kvq_internal.h"],
-                  "decode_mma_kernel": ["kvq_decode_mma.cu", "kvq_decode.cuh", "kvq_common.cuh", "kvq_internal.h"]}
 
 
 def src_hash(kernel: str):
@@ -74,36 +87,85 @@ def profiled_traffic(kernel: str, workload: str):
     return None
 
 
-# --------------------------------------------------------------------------- workload
+# --------------------------------------------------------------------------- workloads
 
 class Workload:
+    """Device-resident inputs of one serving step, plus the untimed prefill that precedes it."""
+
     def __init__(self, name: str, seed: int, device):
-        self.wl = synth.WORKLOADS[name]
-        self.name = name
-        self.lengths = synth.seq_lengths(name, seed=seed)
-        self.T = sum(self.lengths)
-        self.B = len(self.lengths)
-        self.H, self.Hq, self.ps = self.wl.num_kv_heads, self.wl.num_q_heads, self.wl.page_size
-        # inputs below 1 GB are drawn on the CPU (identical on every machine), larger ones on the device
-        gen_dev = "cpu" if self.T * self.H * 128 * 2 * 2 < (1 << 30) or device.type == "cpu" else device
-        self.k, self.v = (t.to(device) for t in synth.make_kv(self.T, self.wl, seed, device=gen_dev, chunk=8192))
-        pt, self.num_pages = synth.make_page_table(self.lengths, self.ps, seed)
+        wl = synth.WORKLOADS[name]
+        self.wl, self.name, self.seed, self.device = wl, name, seed, device
+        self.H, self.Hq, self.ps = wl.num_kv_heads, wl.num_q_heads, wl.page_size
+        lengths = synth.seq_lengths(name, seed=seed)
+        self.lengths = lengths
+        B = len(lengths)
+        if name in ("batch16", "single256"):
+            self.prefill = []  # (sequence lengths, starts) appended untimed
+            step = [(lengths, [0] * B)]
+            dec_seqs, dec_lens = list(range(B)), lengths
+            caps = lengths
+        elif name == "decode64x8k":
+            self.prefill = [(lengths, [0] * B)]
+            step = [([1] * B, lengths)]
+            dec_seqs, dec_lens = list(range(B)), [L + 1 for L in lengths]
+            caps = [L + 1 for L in lengths]
+        elif name == "mixed256":
+            rng = np.random.default_rng(seed + 7)
+            prefilling = set(rng.choice(B, 8, replace=False).tolist())
+            self.prefill = [(lengths, [0] * B)]
+            step = [([2048 if s in prefilling else 1 for s in range(B)], lengths)]
+            dec_seqs = [s for s in range(B) if s not in prefilling]
+            dec_lens = [lengths[s] + 1 for s in dec_seqs]
+            caps = [L + 2048 for L in lengths]
+        elif name == "long1m":
+            L = lengths[0]
+            self.prefill = []
+            step = [([8192], [c]) for c in range(0, L, 8192)]
+            dec_seqs, dec_lens = [0], [L]
+            caps = lengths
+        else:
+            raise KeyError(name)
+        pt, self.num_pages = synth.make_page_table(caps, self.ps, seed)
         self.page_table = pt.to(device)
-        ts, tp = synth.append_positions(self.lengths)
-        self.tok_seq, self.tok_pos = ts.to(device), tp.to(device)
-        self.q = synth.make_q(self.B, self.Hq, 128, seed).to(device)
-        self.seq_lens = torch.tensor(self.lengths, dtype=torch.int32, device=device)
-        self.max_len = max(self.lengths)
+        self.pt_stride, self.num_seqs = pt.shape[1], pt.shape[0]
+        # the step's appends: one call per entry, each with its own tokens
+        self.appends = []
+        for i, (ls, st) in enumerate(step):
+            ts, tp = synth.append_positions(ls, st)
+            k, v = self._rows(len(ts), 1000 + i)
+            self.appends.append((k, v, ts.to(device), tp.to(device)))
+        self.tokens_per_step = sum(int(a[2].numel()) for a in self.appends)
+        self.dec_lens = dec_lens
+        self.dec_B = len(dec_seqs)
+        self.dec_pt = pt[dec_seqs].contiguous().to(device)
+        self.q = synth.make_q(self.dec_B, self.Hq, 128, seed).to(device)
+        self.seq_lens = torch.tensor(dec_lens, dtype=torch.int32, device=device)
+        self.max_len = max(dec_lens)
+
+    def _rows(self, n, salt):
+        # inputs below 1 GB are drawn on the CPU (identical on every machine), larger ones on the device
+        gen = "cpu" if n * self.H * 128 * 2 * 2 < (1 << 30) or self.device.type == "cpu" else self.device
+        k, v = synth.make_kv(n, self.wl, self.seed * 7 + salt, device=gen, chunk=8192)
+        return k.to(self.device), v.to(self.device)
+
+    def run_prefill(self, cache):
+        for i, (ls, st) in enumerate(self.prefill):
+            ts, tp = synth.append_positions(ls, st)
+            for c0 in range(0, len(ts), 1 << 20):
+                c1 = min(len(ts), c0 + (1 << 20))
+                k, v = self._rows(c1 - c0, 10_000 + i * 4096 + c0 // (1 << 20))
+                cache.append(k, v, ts[c0:c1].to(self.device), tp[c0:c1].to(self.device), self.page_table)
+                del k, v
 
     def append_bytes(self, mode):
         # read K and V rows (2 x 256 B per head); write bf16 rows (2 x 256 B) or INT4 codes + scale/zero (2 x 68 B)
         write = 2 * 256 if mode == kvq.KV_BF16 else 2 * 68
-        return self.T * self.H * (2 * 256 + write)
+        return self.tokens_per_step * self.H * (2 * 256 + write)
 
     def decode_bytes(self, mode):
         per_tok = self.H * (2 * 256 if mode == kvq.KV_BF16 else 2 * 68)
-        pages = sum(-(-L // self.ps) for L in self.lengths)
-        return self.T * per_tok + self.B * self.Hq * 128 * 2 * 2 + pages * 4
+        pages = sum(-(-L // self.ps) for L in self.dec_lens)
+        return sum(self.dec_lens) * per_tok + self.dec_B * self.Hq * 128 * 2 * 2 + pages * 4
 
 
 class ClockSampler:
@@ -152,24 +214,28 @@ class ClockSampler:
 
 
 def make_cache(w: Workload, mode, b, rv, device):
-    return kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0)
+    cache = kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0)
+    w.run_prefill(cache)
+    return cache
 
 
 def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False):
-    """Device-timed steps; returns per-kernel and per-step mean times (ms)."""
+    """Device-timed steps (CUDA events on the launching stream); per-kernel and per-step means (ms)."""
     cache = make_cache(w, mode, b, rv, device)
-    ws, _ = cache.workspace(w.B, w.max_len, device)
-    out = torch.empty(w.B, w.Hq, 128, dtype=torch.bfloat16, device=device)
+    ws, _ = cache.workspace(w.dec_B, w.max_len, device)
+    out = torch.empty(w.dec_B, w.Hq, 128, dtype=torch.bfloat16, device=device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
 
     def step(e=None):
         if e: e[0].record(stream)
-        cache.append(w.k, w.v, w.tok_seq, w.tok_pos, w.page_table, stream)
+        for k, v, ts, tp in w.appends:
+            kvq.kv_append_quant(cache.handle, k, v, k.shape[0], ts, tp, w.page_table, w.pt_stride, w.num_seqs,
+                                stream)
         if e: e[1].record(stream)
-        kvq.kv_decode_attn(cache.handle, w.q, w.seq_lens, w.page_table, w.page_table.shape[1], w.B, w.max_len,
-                           out, 0, ws, ws.numel(), stream)
+        kvq.kv_decode_attn(cache.handle, w.q, w.seq_lens, w.dec_pt, w.pt_stride, w.dec_B, w.max_len, out, 0, ws,
+                           ws.numel(), stream)
         if e: e[2].record(stream)
 
     for _ in range(warmup):
@@ -200,30 +266,35 @@ def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False):
     cache.close()
     return {"append_ms": float(app.mean()), "decode_ms": float(dec.mean()), "step_ms": float((app + dec).mean()),
             "append_ms_median": float(np.median(app)), "decode_ms_median": float(np.median(dec)),
-            "wall_s": wall, "status": status, "clocks": sampler.summary() if sampler else None}
+            "wall_s": wall, "status": status, "clocks": sampler.summary() if sampler else None,
+            "launches_per_step": len(w.appends) + 2}
 
 
 def run_e2e(w: Workload, mode, b, rv, steps, warmup, device):
     """Same step through the C ABI with pinned HOST inputs: H2D copies of the step's inputs and a
-    D2H read of the attention output are inside the timed region."""
+    D2H read of the attention output are inside the timed region (CUDA events, launching stream)."""
     cache = make_cache(w, mode, b, rv, device)
-    ws, _ = cache.workspace(w.B, w.max_len, device)
-    host = {n: getattr(w, n).cpu().pin_memory() for n in ("k", "v", "tok_seq", "tok_pos", "page_table", "q",
-                                                          "seq_lens")}
-    dev = {n: torch.empty_like(t, device=device) for n, t in host.items()}
-    out = torch.empty(w.B, w.Hq, 128, dtype=torch.bfloat16, device=device)
+    ws, _ = cache.workspace(w.dec_B, w.max_len, device)
+    host = [[t.cpu().pin_memory() for t in a] for a in w.appends]
+    hdec = [t.cpu().pin_memory() for t in (w.q, w.seq_lens, w.dec_pt, w.page_table)]
+    dev = [[torch.empty_like(t, device=device) for t in a] for a in host]
+    ddec = [torch.empty_like(t, device=device) for t in hdec]
+    out = torch.empty(w.dec_B, w.Hq, 128, dtype=torch.bfloat16, device=device)
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     stream = torch.cuda.current_stream(device)
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = sum(t.numel() * t.element_size() for a in host for t in a) + sum(t.numel() * t.element_size() for t in hdec)
     d2h = out_h.numel() * out_h.element_size()
 
     def step():
-        for n, t in host.items():
-            dev[n].copy_(t, non_blocking=True)
-        kvq.kv_append_quant(cache.handle, dev["k"], dev["v"], w.T, dev["tok_seq"], dev["tok_pos"],
-                            dev["page_table"], w.page_table.shape[1], w.B, stream)
-        kvq.kv_decode_attn(cache.handle, dev["q"], dev["seq_lens"], dev["page_table"], w.page_table.shape[1],
-                           w.B, w.max_len, out, 0, ws, ws.numel(), stream)
+        for hd, dd in zip(hdec, ddec):
+            dd.copy_(hd, non_blocking=True)
+        q, sl, dpt, pt = ddec
+        for ha, da in zip(host, dev):
+            for h_, d_ in zip(ha, da):
+                d_.copy_(h_, non_blocking=True)
+            k, v, ts, tp = da
+            kvq.kv_append_quant(cache.handle, k, v, k.shape[0], ts, tp, pt, w.pt_stride, w.num_seqs, stream)
+        kvq.kv_decode_attn(cache.handle, q, sl, dpt, w.pt_stride, w.dec_B, w.max_len, out, 0, ws, ws.numel(), stream)
         out_h.copy_(out, non_blocking=True)
 
     for _ in range(warmup):
@@ -244,18 +315,19 @@ def run_e2e(w: Workload, mode, b, rv, steps, warmup, device):
 
 # --------------------------------------------------------------------------- oracle (CPU)
 
-def oracle_inputs(w: Workload):
-    bits = lambda t: t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-    return dict(k=bits(w.k), v=bits(w.v), q=bits(w.q), ts=w.tok_seq.cpu().numpy(), tp=w.tok_pos.cpu().numpy(),
-                pt=w.page_table.cpu().numpy())
-
-
-def oracle_step_estimate(w: Workload, inp, mode, b, rv, tok_budget: int, row_budget: int):
-    """Run the oracle on a bounded sample (the first tok_budget tokens appended, row_budget
-    decode rows) and return (seconds one full step would take, sample description)."""
+def oracle_unit_costs(w: Workload, mode, b, rv, tok_budget: int, row_budget: int, seed=0):
+    """Seconds per appended token and per (cached token x query head) of the CPU oracle, measured
+    on a bounded sample shaped like the workload (tok_budget appended tokens; row_budget decode
+    rows over a sequence of the workload's mean decoded length)."""
     import oracle
 
-    H, ps, P = w.H, w.ps, w.num_pages
+    H, ps = w.H, w.ps
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    n = max(1, tok_budget)
+    k, v = synth.make_kv(n, w.wl, seed)
+    Ls = int(min(max(np.mean(w.dec_lens), 16), 32768))
+    cap = max(n, Ls)
+    pt, P = synth.make_page_table([cap], ps, seed)
     if mode == kvq.KV_BF16:
         kp = np.zeros((P, H, ps, 128), np.uint16)
         ks = np.zeros(1, np.uint16)
@@ -263,21 +335,24 @@ def oracle_step_estimate(w: Workload, inp, mode, b, rv, tok_budget: int, row_bud
         kp = np.zeros((P, H, ps, 64), np.uint8)
         ks = np.zeros((P, H, ps, 2), np.uint16)
     vp, vs = kp.copy(), ks.copy()
-    n = max(1, min(tok_budget, w.T))
+    ts, tp = synth.append_positions([n])
     t0 = time.perf_counter()
-    oracle.append(mode, b, rv, kp, vp, ks, vs, inp["k"][:n], inp["v"][:n], inp["ts"][:n], inp["tp"][:n], inp["pt"])
-    t_app = time.perf_counter() - t0
-    rows_all = [(s, j) for s in range(w.B) for j in range(w.Hq)]
-    rng = np.random.default_rng(0)
-    r = max(1, min(row_budget, len(rows_all)))
-    pick = [rows_all[i] for i in sorted(rng.choice(len(rows_all), r, replace=False))]
+    oracle.append(mode, b, rv, kp, vp, ks, vs, bits(k), bits(v), ts.numpy(), tp.numpy(), pt.numpy())
+    c_app = (time.perf_counter() - t0) / n
+    q = synth.make_q(1, w.Hq, 128, seed)
+    r = max(1, min(row_budget, w.Hq))
+    rows = [(0, j) for j in range(r)]
     t0 = time.perf_counter()
-    oracle.decode(mode, b, rv, kp, vp, ks, vs, inp["q"], np.array(w.lengths), inp["pt"], H, rows=pick)
-    t_dec = time.perf_counter() - t0
-    est = t_app * (w.T / n) + t_dec * (len(rows_all) / r)
-    sample = f"oracle append of {n}/{w.T} tokens + decode of {r}/{len(rows_all)} (seq, q-head) rows, " \
-             f"1 thread, scaled to one full step"
-    return est, sample
+    oracle.decode(mode, b, rv, kp, vp, ks, vs, bits(q), np.array([Ls]), pt.numpy(), H, rows=rows)
+    c_dec = (time.perf_counter() - t0) / (r * Ls)
+    sample = (f"oracle append of {n} tokens and decode of {r} query-head rows over {Ls} cached tokens, "
+              f"1 thread; per-unit costs scaled to one step ({w.tokens_per_step} tokens appended, "
+              f"{sum(w.dec_lens) * w.Hq} (token x query head) decoded)")
+    return c_app, c_dec, sample
+
+
+def oracle_step_seconds(w: Workload, c_app, c_dec):
+    return c_app * w.tokens_per_step + c_dec * sum(w.dec_lens) * w.Hq
 
 
 # --------------------------------------------------------------------------- dist
@@ -293,7 +368,8 @@ def _init_dist():
 
         import torch.distributed as dist
 
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         _dist = dist
     return ws
 
@@ -303,19 +379,12 @@ def _barrier():
         _dist.barrier()
 
 
-def max_over_ranks(x: float, device) -> float:
+def reduce_over_ranks(x: float, op: str, device) -> float:
+    """MAX or SUM of one number over all ranks (the only collectives: timing bookkeeping)."""
     if _dist is None:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=device)
-    _dist.all_reduce(t, op=_dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def sum_over_ranks(x: float, device) -> float:
-    if _dist is None:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device=device)
-    _dist.all_reduce(t, op=_dist.ReduceOp.SUM)
+    _dist.all_reduce(t, op=_dist.ReduceOp.MAX if op == "max" else _dist.ReduceOp.SUM)
     return float(t.item())
 
 
@@ -324,7 +393,7 @@ def sum_over_ranks(x: float, device) -> float:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default="batch16", choices=list(synth.WORKLOADS))
@@ -343,33 +412,32 @@ def main():
     world = _init_dist()
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    w = Workload(args.workload, args.seed + rank, device)
+    w = Workload(args.workload, args.seed + rank, device)  # each rank: its own independent batch
+    hname, hmode, hb, hrv = HEADLINE[args.workload]
 
-    res = run_variant(w, kvq.KV_INT4_BDR, 128, False, args.steps, args.warmup, device, clocks=True)
-    step_ms = max_over_ranks(res["step_ms"], device)
-    tokens = sum_over_ranks(w.T, device)
+    res = run_variant(w, hmode, hb, hrv, args.steps, args.warmup, device, clocks=True)
+    step_ms = reduce_over_ranks(res["step_ms"], "max", device)
+    tokens = reduce_over_ranks(w.tokens_per_step, "sum", device)
     value = tokens / (step_ms / 1e3)
 
     sweep = {}
-    if not args.no_sweep:
+    if not args.no_sweep and args.workload == "batch16":
         n = max(50, min(args.steps // 4, 500))
         for name, mode, b, rv in VARIANTS:
-            r = res if name == HEADLINE else run_variant(w, mode, b, rv, n, 3, device)
-            sweep[name] = {"append_tok_per_s": w.T / (r["append_ms"] / 1e3),
+            r = res if name == hname else run_variant(w, mode, b, rv, n, 3, device)
+            sweep[name] = {"append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
                            "append_gbs": w.append_bytes(mode) / (r["append_ms"] / 1e3) / 1e9,
                            "decode_gbs": w.decode_bytes(mode) / (r["decode_ms"] / 1e3) / 1e9,
                            "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3}
-        if "int4" in sweep:
-            sweep["bdr128_k_over_int4_append"] = sweep[HEADLINE]["append_tok_per_s"] / sweep["int4"]["append_tok_per_s"]
+        sweep["bdr128_k_over_int4_append"] = sweep["bdr128_k"]["append_tok_per_s"] / sweep["int4"]["append_tok_per_s"]
 
-    e2e_ms, h2d, d2h = run_e2e(w, kvq.KV_INT4_BDR, 128, False, max(20, args.steps // 20), args.warmup, device)
-    e2e_ms = max_over_ranks(e2e_ms, device)
+    e2e_ms, h2d, d2h = run_e2e(w, hmode, hb, hrv, max(20, min(200, args.steps // 20)), args.warmup, device)
+    e2e_ms = reduce_over_ranks(e2e_ms, "max", device)
 
     peak, peak_kind = peak_hbm()
-    app_b, dec_b = w.append_bytes(kvq.KV_INT4_BDR), w.decode_bytes(kvq.KV_INT4_BDR)
+    app_b, dec_b = w.append_bytes(hmode), w.decode_bytes(hmode)
     app_gbs = app_b / (res["append_ms"] / 1e3) / 1e9
     dec_gbs = dec_b / (res["decode_ms"] / 1e3) / 1e9
     dominant = "append" if res["append_ms"] >= res["decode_ms"] else "decode"
@@ -379,36 +447,37 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 in, int4+fp16 scale/zero cache, fp32 math", "data": "synthetic",
-        "config": {"workload": args.workload, "description": w.wl.description, "variant": "INT4+BDR-128, keys only",
-                   "sequences": w.B, "tokens_appended_per_step": w.T, "cached_tokens_decoded_per_step": w.T,
+        "vs_baseline": None, "dtype": "bf16 in, int4 codes + fp16 scale/zero cache, fp32 math", "data": "synthetic",
+        "config": {"workload": args.workload, "description": w.wl.description, "variant": hname,
+                   "sequences": len(w.lengths), "tokens_appended_per_step": w.tokens_per_step,
+                   "sequences_decoded_per_step": w.dec_B, "cached_tokens_decoded_per_step": sum(w.dec_lens),
                    "num_kv_heads": w.H, "num_q_heads": w.Hq, "head_dim": 128, "page_size": w.ps,
                    "l2": "256 MiB buffer written between timed steps (L2 is 126 MB)",
                    "parallelism": f"{world} independent replica(s), one per GPU, no collective on the data path",
                    "seed": args.seed},
         "components": {
-            "append": {"us": res["append_ms"] * 1e3, "tokens_per_s": w.T / (res["append_ms"] / 1e3),
+            "append": {"us": res["append_ms"] * 1e3, "tokens_per_s": w.tokens_per_step / (res["append_ms"] / 1e3),
                        "algorithmic_bytes": app_b, "gbs": app_gbs, "frac_of_peak": app_gbs / peak,
-                       "frac_of_8tbs": app_gbs / NOMINAL_HBM_GBS},
+                       "frac_of_8tbs": app_gbs / NOMINAL_HBM_GBS, "launches_per_step": len(w.appends)},
             "decode": {"us": res["decode_ms"] * 1e3, "algorithmic_bytes": dec_b, "gbs": dec_gbs,
                        "frac_of_peak": dec_gbs / peak, "frac_of_8tbs": dec_gbs / NOMINAL_HBM_GBS,
-                       "note": "split + merge kernels; reads the pages the append of the same step wrote"}},
+                       "note": "split + merge kernels"}},
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
                      "frac": dom_gbs / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                      "traffic": traffic},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": res["launches_per_step"] * args.steps,
         "clocks": res["clocks"],
         "device_status": kvq.status_string(res["status"]),
     }
     if sweep:
         line["sweep"] = sweep
     if rank == 0 and world == 1 and not args.no_cpu:
-        inp = oracle_inputs(w)
-        est, sample = oracle_step_estimate(w, inp, kvq.KV_INT4_BDR, 128, False, tok_budget=w.T, row_budget=96)
-        line["cpu_baseline"] = {"value": w.T / est, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": sample}
+        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=min(w.tokens_per_step, 20000),
+                                                 row_budget=8)
+        line["cpu_baseline"] = {"value": w.tokens_per_step / oracle_step_seconds(w, c_app, c_dec),
+                                "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if _dist is not None:
@@ -416,28 +485,28 @@ def main():
 
 
 def run_reference(args, world):
-    """The CPU oracle as the reference arm, on a bounded sample per step (rank 0 only)."""
+    """The CPU oracle as the reference arm (rank 0 only): each step runs a bounded sample of the
+    workload's step on the host cores and scales its unit costs to the full step."""
     w = Workload(args.workload, args.seed, torch.device("cpu"))
-    inp = oracle_inputs(w)
+    _, hmode, hb, hrv = HEADLINE[args.workload]
     budget_s = 120.0
-    per_step = budget_s / (args.steps + args.warmup)
-    # calibrate: seconds per token (append) and per row (decode)
-    est0, _ = oracle_step_estimate(w, inp, kvq.KV_INT4_BDR, 128, False, tok_budget=256, row_budget=2)
-    frac = min(1.0, per_step / max(est0, 1e-9))
-    tok = max(16, int(w.T * frac))
-    rows = max(1, int(w.B * w.Hq * frac))
+    c_app, c_dec, _ = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=256, row_budget=1)
+    unit = max(oracle_step_seconds(w, c_app, c_dec), 1e-9)
+    frac = min(1.0, budget_s / (args.steps + args.warmup) / unit)
+    tok = max(16, int(min(w.tokens_per_step, 20000) * frac))
+    rows = max(1, int(8 * frac))
     times, sample = [], ""
     for i in range(args.warmup + args.steps):
-        est, sample = oracle_step_estimate(w, inp, kvq.KV_INT4_BDR, 128, False, tok_budget=tok, row_budget=rows)
+        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=tok, row_budget=rows, seed=i)
         if i >= args.warmup:
-            times.append(est)
+            times.append(oracle_step_seconds(w, c_app, c_dec))
     step_s = float(np.mean(times))
-    value = w.T / step_s
+    value = w.tokens_per_step / step_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 write path, f64 attention", "data": "synthetic",
-            "config": {"workload": args.workload, "variant": "INT4+BDR-128, keys only", "sequences": w.B,
-                       "tokens_appended_per_step": w.T},
+            "config": {"workload": args.workload, "variant": HEADLINE[args.workload][0],
+                       "sequences": len(w.lengths), "tokens_appended_per_step": w.tokens_per_step},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
