@@ -92,12 +92,12 @@ __global__ void __launch_bounds__(kThreads) bf16_split_kernel(Params p) {
         bool valid = t < t1;
         int64_t row = 0;
         if (valid) {
-            const int page = __ldg(pt + t / ps);
+            const int page = __ldg(pt + page_of_pos(p, t));
             if (page < 0 || page >= p.g.num_pages) {
                 flag_error(p.err, kErrOOB);
                 valid = false;
             } else {
-                row = (int64_t(page) * H + h) * ps + (t % ps);
+                row = (int64_t(page) * H + h) * ps + slot_of_pos(p, t);
             }
         }
         float sc[G];
@@ -285,11 +285,14 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
 DecodePlan plan_decode(const CacheGeom& g, int batch, int max_seq_len, int num_sms) {
-    // Items of a multiple of 64 tokens (4 warps x 16-token chunks), at least 256 and at
-    // most 8192 tokens, sized so a full batch at the length bound makes ~2048 items.
+    // Splits of a multiple of 64 tokens (4 warps x 16-token chunks), between 256 and 8192
+    // tokens (bounding how many steps one warp accumulates), sized so that a full batch at the length bound gives about 2.5 waves of
+    // resident split CTAs (4 per SM): long enough to amortise a CTA's start-up and merge,
+    // short enough to balance the tail.
     DecodePlan pl;
     const int64_t L = max_seq_len > 0 ? max_seq_len : 1;
-    int64_t it = (int64_t(batch) * L + 2047) / 2048;
+    const int64_t slots = int64_t(num_sms > 0 ? num_sms : 148) * 4;
+    int64_t it = (int64_t(batch) * g.H * L * 2 + 5 * slots - 1) / (5 * slots);
     it = ((it + 63) / 64) * 64;
     if (it < 256) it = 256;
     if (it > 8192) it = 8192;
@@ -313,6 +316,9 @@ cudaError_t launch_decode(const CacheGeom& g, const DecodeArgs& a, const DecodeP
     p.item_tokens = plan.item_tokens;
     p.max_splits = plan.max_splits;
     p.qscale = float(1.0 / sqrt(double(kHeadDim))) * kLog2e;
+    p.ps_shift = -1;
+    for (int sh = 0; sh < 11; ++sh)
+        if ((1 << sh) == g.page_size) p.ps_shift = sh;
     p.ws_o = reinterpret_cast<float*>(ws);
     p.ws_ml = reinterpret_cast<float2*>(ws + align256(rows * kHeadDim * sizeof(float)));
     p.err = err_word;

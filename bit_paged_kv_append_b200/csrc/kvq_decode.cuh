@@ -27,6 +27,7 @@ struct DecodeParams {
     int item_tokens;  // cached tokens per split, a multiple of 64
     int max_splits;   // ceil(max_seq_len / item_tokens), >= 1
     float qscale;     // 1/sqrt(D) * log2(e): scores live in the log2 domain
+    int ps_shift;     // log2(page_size) when it is a power of two, else -1
     float* ws_o;      // [B][max_splits][Hq][D] unnormalised partial outputs
     float2* ws_ml;    // [B][max_splits][Hq] (running max, sum of weights)
     int* err;
@@ -52,6 +53,14 @@ __device__ __forceinline__ int decode_len(const DecodeParams& p, int s) {
     const int L = __ldg(p.a.seq_lens + s);
     const int cap = min(p.a.pt_stride * p.g.page_size, p.a.max_seq_len);
     return L < 0 ? 0 : (L > cap ? cap : L);
+}
+
+// Page-table index and slot of token position t (shifts for power-of-two page sizes).
+__device__ __forceinline__ int page_of_pos(const DecodeParams& p, int t) {
+    return p.ps_shift >= 0 ? (t >> p.ps_shift) : t / p.g.page_size;
+}
+__device__ __forceinline__ int slot_of_pos(const DecodeParams& p, int t) {
+    return p.ps_shift >= 0 ? (t & (p.g.page_size - 1)) : t % p.g.page_size;
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {  // MUFU ex2; exp2(-inf) = +0

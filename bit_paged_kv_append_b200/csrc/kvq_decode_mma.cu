@@ -26,12 +26,14 @@
 //     whose A entries carry a factor 1/16): one AND per two codes, no bias to
 //     cancel, every product exact; the scores are scaled back by 2^24.
 //   * P.V: D[16 dims x 8 heads] = A[16 x 16 tokens] B[16 tokens x 8 heads].  A =
-//     V codes of four tokens (PRMT + AND), B = p * scale_v, taken straight from
-//     the q.K accumulator layout (the thread that holds a score also holds
-//     the matching B element), so no shuffle or transpose.  B is split into
-//     fp16 high and low parts accumulated by two mmas: sum (p scale) c and
-//     sum p zero nearly cancel, so a single fp16 rounding of p * scale would
-//     cost ~1e-3 of the output.
+//     V codes of four tokens (PRMT + AND), centred to c - 8 by one exact fp16
+//     add, B = p * scale_v, taken straight from the q.K accumulator layout (the
+//     thread that holds a score also holds the matching B element), so no
+//     shuffle or transpose.  Centring keeps the accumulator small: the tensor
+//     cores' fp32 accumulation does not round to nearest, and over thousands of
+//     tokens sum (p scale) c and sum p zero would otherwise nearly cancel.  B
+//     is split into fp16 high and low parts accumulated by two mmas, since a
+//     single fp16 rounding of p * scale would cost ~1e-3 of the output.
 //   * Which dimension d and which token each fragment slot stands for is a
 //     fixed permutation chosen so every thread reads contiguous bytes and the
 //     shared-memory reads are conflict-free; the output mapping undoes it.
@@ -79,6 +81,15 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
 }
+
+// fp16x2 add of raw words (exact here: every operand and sum is a small multiple of 2^-24)
+__device__ __forceinline__ uint32_t hadd2u(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+constexpr uint32_t kMinus8 = 0x80088008u;    // fp16x2 (-8 2^-24, -8 2^-24)
+constexpr uint32_t kMinus128 = 0x80808080u;  // fp16x2 (-128 2^-24, -128 2^-24)
 
 __device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half(uint16_t(w & 0xFFFF))); }
 __device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half(uint16_t(w >> 16))); }
@@ -131,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         if ((iw >> 5) != win) {
             win = iw >> 5;
             const int ci = 32 * win + lane;
-            mypage = ci < nw ? __ldg(pt + (t0 + (warp + kWarps * ci) * kChunk) / ps) : -1;
+            mypage = ci < nw ? __ldg(pt + page_of_pos(p, t0 + (warp + kWarps * ci) * kChunk)) : -1;
         }
         return __shfl_sync(0xffffffffu, mypage, iw & 31);
     };
@@ -142,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
             const int page = page_of(iw);
             if (lane == 0) {
                 if (page >= 0 && page < p.g.num_pages) {
-                    const int64_t row = (int64_t(page) * H + h) * ps + (tb % ps);
+                    const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, tb);
                     smask[warp][slot] = 0xFFFFu;
                     fence_proxy_async();
                     mbar_expect_tx(&bars[warp][slot], kStageBytes);
@@ -163,10 +174,10 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
             const int t = tb + i;
             bool ok = false;
             if (t < t1) {
-                const int page = __ldg(pt + t / ps);
+                const int page = __ldg(pt + page_of_pos(p, t));
                 ok = page >= 0 && page < p.g.num_pages;
                 if (ok) {
-                    const int64_t row = (int64_t(page) * H + h) * ps + (t % ps);
+                    const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, t);
                     const uint4* src = reinterpret_cast<const uint4*>((isv ? vpool : kpool) + row * 64);
                     uint4* dst = reinterpret_cast<uint4*>(st + (isv ? kOffV : 0) + i * 64);
 #pragma unroll
@@ -262,7 +273,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         const int tb = t0 + (warp + kWarps * i) * kChunk;
         {  // each lane converts one (scale, zero) word: lanes 0..15 K, 16..31 V
             const uint32_t w = reinterpret_cast<const uint32_t*>(st + kOffKs)[lane];
-            szf[warp][lane >> 4][lane & 15] = make_float2(half_lo(w), half_hi(w));
+            const float sc = half_lo(w), zr = half_hi(w);
+            // values use centred codes c - 8, so their offset is zero + 8 scale
+            szf[warp][lane >> 4][lane & 15] = make_float2(sc, lane < 16 ? zr : zr + 8.0f * sc);
             __syncwarp();
         }
 
@@ -352,8 +365,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
 #pragma unroll
                 for (int sh = 0; sh < 2; ++sh) {
                     const int jv = 4 * wq + 2 * bp + sh;  // byte of the thread's 8-byte slice
-                    const uint32_t a[4] = {P0 & 0x000F000Fu, P0 & 0x00F000F0u, P1 & 0x000F000Fu,
-                                           P1 & 0x00F000F0u};
+                    // centred codes (c - 8) 2^-24 and 16 (c - 8) 2^-24: exact subnormal fp16
+                    const uint32_t a[4] = {hadd2u(P0 & 0x000F000Fu, kMinus8), hadd2u(P0 & 0x00F000F0u, kMinus128),
+                                           hadd2u(P1 & 0x000F000Fu, kMinus8), hadd2u(P1 & 0x00F000F0u, kMinus128)};
                     mma16816(O[jv], a, b0, b1);
                     mma16816(O[jv], a, b0l, b1l);
                     P0 >>= 8;
