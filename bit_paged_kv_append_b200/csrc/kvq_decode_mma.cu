@@ -1,41 +1,49 @@
 // kvq_decode_mma.cu -- paged GQA decode attention over the INT4 cache on the
-// tensor cores (mma.sync m16n8k16, fp16 operands, fp32 accumulation).
+// tensor cores (mma.sync: int8 and fp16 operands, int32 / fp32 accumulation).
 //
 // SAW-INT4 (wispaper.ai blog, section 3): the query is rotated in step with
 // H_blk, so q' k^ needs no inverse rotation of the cache; the abstract keeps
 // fused attention over the paged INT4 layout.  Dequantisation is factored:
 //   q' . (scale c + zero) = scale (q' . c) + zero sum(q')
 //   sum_t p_t (scale_t c_t + zero_t) = sum_t (p_t scale_t) c_t + sum_t p_t zero_t
-// so both contractions run on raw 4-bit codes, which are exact in fp16.
+// so both contractions run on raw 4-bit codes.
 //
 // One CTA = (split, KV head, sequence), 4 warps; each warp walks 16-token
 // chunks of its split (round robin), with its own online-softmax state.  The
-// CTA issues its first copies before anything else, then rotates q (one warp
-// per head, FWHT with shuffles) straight into mma fragment order, so the
+// CTA issues its first copies before anything else, then prepares q, so the
 // prologue hides under the first memory latency.
 //   * Staging: per warp a ring of 4 shared-memory stages; one lane issues 1-D
 //     bulk async copies (cp.async.bulk, no multicast) of the chunk's K codes,
 //     V codes and scale/zero words (2176 B) on an mbarrier; every wait is
 //     bounded.  Page sizes that are not a multiple of 16 take a per-token
 //     gather instead.
-//   * q.K: D[16 x 8] = A[16 x 16] B[16 x 8] per (n-tile of 8 tokens, 16 dims).
-//     A = the G rotated query heads, each split into an fp16 high part (rows
-//     0..7) and low part (rows 8..15), so q' keeps ~22 bits; B = codes.  A
-//     code nibble c is masked in place into an fp16 lane, which makes it the
-//     exact subnormal c * 2^-24 (16 c * 2^-24 for the high nibble of a byte,
-//     whose A entries carry a factor 1/16): one AND per two codes, no bias to
-//     cancel, every product exact; the scores are scaled back by 2^24.
-//   * P.V: D[16 dims x 8 heads] = A[16 x 16 tokens] B[16 tokens x 8 heads].  A =
-//     V codes of four tokens (PRMT + AND), centred to c - 8 by one exact fp16
-//     add, B = p * scale_v, taken straight from the q.K accumulator layout (the
-//     thread that holds a score also holds the matching B element), so no
-//     shuffle or transpose.  Centring keeps the accumulator small: the tensor
-//     cores' fp32 accumulation does not round to nearest, and over thousands of
-//     tokens sum (p scale) c and sum p zero would otherwise nearly cancel.  B
-//     is split into fp16 high and low parts accumulated by two mmas, since a
-//     single fp16 rounding of p * scale would cost ~1e-3 of the output.
-//   * Which dimension d and which token each fragment slot stands for is a
-//     fixed permutation chosen so every thread reads contiguous bytes and the
+//   * P.V (both tiles): D[16 dims x 8 cols] += A[16 dims x 16 tokens] B[16 tokens
+//     x 8 cols].  A = V codes of two tokens per register (PRMT + AND) masked
+//     into fp16 lanes, where a nibble c is the exact subnormal c 2^-24, and
+//     centred to c - 8 by one exact fp16 add.  Centring keeps the accumulator
+//     small: the tensor cores' fp32 accumulation does not round to nearest, and
+//     over thousands of tokens sum (p scale) c and sum p zero would otherwise
+//     nearly cancel.  B = p scale_v as an fp16 high part plus an fp16 low part
+//     (one fp16 rounding of p scale would cost ~1e-3 of the output).
+//
+// Two tiles, by the number G of query heads per KV head:
+//   G = 8, heads on M (decode_mma_kernel): q.K is D[16 x 8 tokens] = A[16 x 16
+//     dims] B[16 dims x 8 tokens] with A = the 8 heads' q' as fp16 high parts
+//     (rows 0..7) and low parts (rows 8..15), B = codes masked in place into
+//     fp16 lanes (one AND per two codes; a high nibble is 16 c 2^-24, so its A
+//     entries carry 1/16).  The score of (head, token) then sits in the thread
+//     that needs it as the P.V B operand; the low part of B is a second mma.
+//   G <= 4, tokens on M (decode_tok_kernel): q.K is D[16 tokens x 8 cols] =
+//     A[16 tokens x 32 dims] B[32 dims x 8 cols] on the int8 tensor path: A =
+//     codes as bytes (AND / shift-AND, 8 codes for 3 instructions), B = q' as
+//     16-bit fixed point per head, split into a signed high and low byte (the
+//     8 columns are 4 heads x {high, low}); the int32 accumulation is exact.
+//     Every lane holds two real scores (no idle rows at G = 4), and the P.V B
+//     operand takes its 8 columns as 4 heads x {high, low part of p scale}, so
+//     the low part costs no extra mma; two shuffles move each score from the
+//     q.K layout to the B layout.
+//   * Which dimension and which token each fragment slot stands for is a fixed
+//     permutation chosen so that every thread reads contiguous bytes and the
 //     shared-memory reads are conflict-free; the output mapping undoes it.
 #include "kvq_common.cuh"
 #include "kvq_decode.cuh"
@@ -54,6 +62,8 @@ constexpr int kOffVs = 2 * kCodeBytes + kChunk * 4;
 constexpr int kStageBytes = 2 * kCodeBytes + 2 * kChunk * 4;  // 2176
 constexpr float kTwo24 = 16777216.0f;  // a masked nibble c in an fp16 lane is the subnormal c * 2^-24
 constexpr float kTwo20 = 1048576.0f;   // ... and a masked high nibble is 16 c * 2^-24 = c * 2^-20
+constexpr int kQFix = 32639;           // |q| fixed point of the int8 tile: 256 hi + lo, hi, lo in [-128, 127]
+constexpr uint32_t kFull = 0xffffffffu;
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
@@ -66,6 +76,15 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
         "{%0, %1, %2, %3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D[16 x 8] += A[16 x 32] (u8) B[32 x 8] (s8), int32 accumulation
+__device__ __forceinline__ void mma16832_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
@@ -94,78 +113,61 @@ constexpr uint32_t kMinus128 = 0x80808080u;  // fp16x2 (-128 2^-24, -128 2^-24)
 __device__ __forceinline__ float half_lo(uint32_t w) { return __half2float(__ushort_as_half(uint16_t(w & 0xFFFF))); }
 __device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ushort_as_half(uint16_t(w >> 16))); }
 
-// Token (within an 8-token n-tile) that column n stands for: the four rows one
+// Token (within an 8-token group) that slot n stands for: the four rows one
 // P.V load touches then fall on both 64-byte halves of the bank space.
 __device__ __forceinline__ int sigma(int n) { return n ^ ((n >> 2) & 1); }
 
-template <int G>
-__global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p) {
-    __shared__ __align__(128) uint8_t ring[kWarps][kStages][kStageBytes];
-    __shared__ __align__(8) uint64_t bars[kWarps][kStages];
-    __shared__ uint32_t smask[kWarps][kStages];
-    __shared__ float2 szf[kWarps][2][kChunk];  // (scale, zero) of the current chunk: [warp][K / V][token]
-    __shared__ uint32_t As[8 * 4 * 32];         // q.K A operand in fragment order: [k-step][reg][lane]
-    __shared__ float qsum_s[kMaxGroup];
+// What a CTA keeps in shared memory for its warps' chunk streams.
+struct CtaRing {
+    uint8_t stage[kWarps][kStages][kStageBytes];
+    uint64_t bars[kWarps][kStages];
+    uint32_t mask[kWarps][kStages];     // tokens of the staged chunk on valid pages (bit per token)
+    float2 szf[kWarps][2][kChunk];      // (scale, offset) of the current chunk: [warp][K / V][token]
+};
 
-    const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int gq = lane >> 2, pq = lane & 3;  // mma group id / thread in group
-    const int H = p.g.H, Hq = p.g.Hq, ps = p.g.page_size;
+// One warp's 16-token chunks of its split: page lookups (one page-table entry per
+// lane, 32 chunks a window) and the copies of chunk iw into a ring stage.
+struct ChunkStream {
+    CtaRing* r;
+    const int32_t* pt;  // this sequence's page-table row
+    int t0, t1, nw, warp, lane, h;
+    bool fast;          // page size a multiple of 16: a chunk is 16 consecutive slots of one page
+    uint64_t pol;
+    int win, mypage;
 
-    const int L = decode_len(p, s);
-    if (k == 0 && h == 0 && tid == 0 && L != __ldg(p.a.seq_lens + s)) flag_error(p.err, kErrOOB);
-    const int t0 = k * p.item_tokens;
-    if (t0 >= L) return;  // past the end of the sequence: no partial (the merge reads only real splits)
-    const int t1 = min(L, t0 + p.item_tokens);
-
-    const bool fast = (ps % kChunk) == 0;
-    const uint8_t* kpool = static_cast<const uint8_t*>(p.g.k_pool);
-    const uint8_t* vpool = static_cast<const uint8_t*>(p.g.v_pool);
-    const uint32_t* ksz = p.g.k_sz;
-    const uint32_t* vsz = p.g.v_sz;
-    const int32_t* pt = p.a.page_table + int64_t(s) * p.a.pt_stride;
-    const int nchunks = (t1 - t0 + kChunk - 1) / kChunk;
-    const int nw = nchunks > warp ? (nchunks - warp + kWarps - 1) / kWarps : 0;  // this warp's chunks
-
-    if (lane == 0) {
-#pragma unroll
-        for (int st = 0; st < kStages; ++st) mbar_init(&bars[warp][st], 1);
-        fence_mbar_init();
-    }
-    for (int w = tid; w < 8 * 4 * 32; w += kThreads) As[w] = 0u;
-    __syncthreads();
-
-    // ---------------- start streaming this warp's chunks ----------------
-    const uint64_t pol = policy_evict_first();
-    int win = -1, mypage = -1;
-    auto page_of = [&](int iw) {  // page of this warp's chunk iw (all lanes; 32 ids per window)
+    __device__ __forceinline__ int page_of(const DecodeParams& p, int iw) {
         if ((iw >> 5) != win) {
             win = iw >> 5;
             const int ci = 32 * win + lane;
             mypage = ci < nw ? __ldg(pt + page_of_pos(p, t0 + (warp + kWarps * ci) * kChunk)) : -1;
         }
-        return __shfl_sync(0xffffffffu, mypage, iw & 31);
-    };
-    auto issue = [&](int iw, int slot) {  // this warp's chunk number iw into ring slot
-        uint8_t* st = ring[warp][slot];
+        return __shfl_sync(kFull, mypage, iw & 31);
+    }
+
+    __device__ __forceinline__ void issue(const DecodeParams& p, int iw, int slot) {
+        uint8_t* st = r->stage[warp][slot];
+        uint64_t* bar = &r->bars[warp][slot];
         const int tb = t0 + (warp + kWarps * iw) * kChunk;
+        const uint8_t* kpool = static_cast<const uint8_t*>(p.g.k_pool);
+        const uint8_t* vpool = static_cast<const uint8_t*>(p.g.v_pool);
+        const int H = p.g.H, ps = p.g.page_size;
         if (fast) {
-            const int page = page_of(iw);
+            const int page = page_of(p, iw);
             if (lane == 0) {
                 if (page >= 0 && page < p.g.num_pages) {
                     const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, tb);
-                    smask[warp][slot] = 0xFFFFu;
+                    r->mask[warp][slot] = 0xFFFFu;
                     fence_proxy_async();
-                    mbar_expect_tx(&bars[warp][slot], kStageBytes);
-                    bulk_g2s(st, kpool + row * 64, kCodeBytes, &bars[warp][slot], pol);
-                    bulk_g2s(st + kOffV, vpool + row * 64, kCodeBytes, &bars[warp][slot], pol);
-                    bulk_g2s(st + kOffKs, ksz + row, kChunk * 4, &bars[warp][slot], pol);
-                    bulk_g2s(st + kOffVs, vsz + row, kChunk * 4, &bars[warp][slot], pol);
+                    mbar_expect_tx(bar, kStageBytes);
+                    bulk_g2s(st, kpool + row * 64, kCodeBytes, bar, pol);
+                    bulk_g2s(st + kOffV, vpool + row * 64, kCodeBytes, bar, pol);
+                    bulk_g2s(st + kOffKs, p.g.k_sz + row, kChunk * 4, bar, pol);
+                    bulk_g2s(st + kOffVs, p.g.v_sz + row, kChunk * 4, bar, pol);
                 } else {
-                    smask[warp][slot] = 0u;
+                    r->mask[warp][slot] = 0u;
                     flag_error(p.err, kErrOOB);
                 }
-                mbar_arrive(&bars[warp][slot]);
+                mbar_arrive(bar);
             }
         } else {
             // gather: lanes 0..15 fetch K rows, lanes 16..31 V rows of tokens tb + (lane & 15)
@@ -182,55 +184,184 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
                     uint4* dst = reinterpret_cast<uint4*>(st + (isv ? kOffV : 0) + i * 64);
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) dst[q4] = __ldg(src + q4);
-                    reinterpret_cast<uint32_t*>(st + (isv ? kOffVs : kOffKs))[i] = __ldg((isv ? vsz : ksz) + row);
+                    reinterpret_cast<uint32_t*>(st + (isv ? kOffVs : kOffKs))[i] =
+                        __ldg((isv ? p.g.v_sz : p.g.k_sz) + row);
                 } else if (!isv) {
                     flag_error(p.err, kErrOOB);
                 }
             }
-            const uint32_t m = __ballot_sync(0xffffffffu, ok) & 0xFFFFu;
+            const uint32_t m = __ballot_sync(kFull, ok) & 0xFFFFu;
             __syncwarp();
             if (lane == 0) {
-                smask[warp][slot] = m;
-                mbar_arrive(&bars[warp][slot]);
+                r->mask[warp][slot] = m;
+                mbar_arrive(bar);
             }
         }
-    };
+    }
+};
+
+// Query row qrow (bf16, 128 dims) as q H_blk * log2(e)/sqrt(D): lane holds dims 4 lane .. 4 lane + 3.
+__device__ __forceinline__ void load_q_rotated(const DecodeParams& p, int64_t qrow, int lane, float (&x)[4]) {
+    const uint2 raw =
+        __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.a.q) + qrow * kHeadDim) + lane);
+    x[0] = __uint_as_float(raw.x << 16);
+    x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(raw.y << 16);
+    x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    float sc = p.qscale;
+    if (p.g.mode == 2) {
+        const int b = p.g.bdr_block;
+        // strides 1 and 2 inside the lane, 4 .. 64 across lanes (lane bit = stride / 4)
+        float y0 = x[0] + x[1], y1 = x[0] - x[1], y2 = x[2] + x[3], y3 = x[2] - x[3];
+        x[0] = y0 + y2;
+        x[2] = y0 - y2;
+        x[1] = y1 + y3;
+        x[3] = y1 - y3;
+        for (int hs = 4; hs < b; hs <<= 1) {
+            const bool upper = (lane & (hs >> 2)) != 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float other = __shfl_xor_sync(kFull, x[c], hs >> 2);
+                x[c] = upper ? other - x[c] : x[c] + other;
+            }
+        }
+        sc *= rsqrtf(float(b));
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) x[c] *= sc;
+}
+
+// Chunk's (scale, zero) words into floats, one word per lane (0..15 K, 16..31 V).
+// Values use centred codes c - 8, so their offset is zero + 8 scale; kscale
+// multiplies the key scales (exactly: a power of two).
+__device__ __forceinline__ void stage_szf(CtaRing& R, const uint8_t* st, int warp, int lane, float kscale) {
+    const uint32_t w = reinterpret_cast<const uint32_t*>(st + kOffKs)[lane];
+    const float sc = half_lo(w), zr = half_hi(w);
+    R.szf[warp][lane >> 4][lane & 15] = lane < 16 ? make_float2(sc * kscale, zr) : make_float2(sc, zr + 8.0f * sc);
+    __syncwarp();
+}
+
+// P.V of one chunk into O[16-dim tile jv][4]: A = V codes of tokens (tokA, tokB),
+// (8 + tokA, 8 + tokB), bytes [8 gq, 8 gq + 8) of each row; row gq of tile jv is
+// dim 16 gq + 2 jv (low nibble), row gq + 8 is dim 16 gq + 2 jv + 1 (high nibble,
+// x16).  With kLow, (b0l, b1l) is accumulated by a second mma with the same A.
+template <bool kLow>
+__device__ __forceinline__ void pv_chunk(float (&O)[8][4], const uint8_t* st, int gq, int tokA, int tokB, uint32_t b0,
+                                         uint32_t b1, uint32_t b0l, uint32_t b1l) {
+    const uint8_t* vc = st + kOffV + 8 * gq;
+    const uint2 v00 = *reinterpret_cast<const uint2*>(vc + tokA * 64);
+    const uint2 v01 = *reinterpret_cast<const uint2*>(vc + tokB * 64);
+    const uint2 v10 = *reinterpret_cast<const uint2*>(vc + (8 + tokA) * 64);
+    const uint2 v11 = *reinterpret_cast<const uint2*>(vc + (8 + tokB) * 64);
+#pragma unroll
+    for (int wq = 0; wq < 2; ++wq) {
+        const uint32_t x00 = wq ? v00.y : v00.x, x01 = wq ? v01.y : v01.x;
+        const uint32_t x10 = wq ? v10.y : v10.x, x11 = wq ? v11.y : v11.x;
+#pragma unroll
+        for (int bp = 0; bp < 2; ++bp) {
+            const uint32_t sel = bp ? 0x7632u : 0x5410u;
+            uint32_t P0 = prmt(x00, x01, sel), P1 = prmt(x10, x11, sel);
+#pragma unroll
+            for (int sh = 0; sh < 2; ++sh) {
+                const int jv = 4 * wq + 2 * bp + sh;  // byte of the thread's 8-byte slice
+                // centred codes (c - 8) 2^-24 and 16 (c - 8) 2^-24: exact subnormal fp16
+                const uint32_t a[4] = {hadd2u(P0 & 0x000F000Fu, kMinus8), hadd2u(P0 & 0x00F000F0u, kMinus128),
+                                       hadd2u(P1 & 0x000F000Fu, kMinus8), hadd2u(P1 & 0x00F000F0u, kMinus128)};
+                mma16816(O[jv], a, b0, b1);
+                if (kLow) mma16816(O[jv], a, b0l, b1l);
+                P0 >>= 8;
+                P1 >>= 8;
+            }
+        }
+    }
+}
+
+// Merge the 4 warps' partial states (mo [warp][G][128] outputs incl. the offset
+// term, mm / ml [warp][G] max and weight sum) and store the split's partial rows.
+template <int G>
+__device__ __forceinline__ void store_partials(const DecodeParams& p, const float* mo, const float* mm,
+                                               const float* ml, int s, int k, int h, int tid) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * G + g]);
+        float acc = 0.0f, lt = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float mw = mm[w * G + g];
+            const float f = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - M);
+            acc += f * mo[(w * G + g) * kHeadDim + tid];
+            lt += f * ml[w * G + g];
+        }
+        const int64_t r = partial_row(p, s, k, h * G + g);
+        p.ws_o[r * kHeadDim + tid] = acc;
+        if (tid == 0) p.ws_ml[r] = make_float2(M, lt);
+    }
+}
+
+// Common start of a CTA: split bounds and the chunk stream.  False: no tokens.
+__device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, ChunkStream& cs, int warp, int lane,
+                                            int tid) {
+    const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int L = decode_len(p, s);
+    if (k == 0 && h == 0 && tid == 0 && L != __ldg(p.a.seq_lens + s)) flag_error(p.err, kErrOOB);
+    const int t0 = k * p.item_tokens;
+    if (t0 >= L) return false;  // past the end of the sequence: no partial (the merge reads only real splits)
+    cs.r = &R;
+    cs.pt = p.a.page_table + int64_t(s) * p.a.pt_stride;
+    cs.t0 = t0;
+    cs.t1 = min(L, t0 + p.item_tokens);
+    const int nchunks = (cs.t1 - t0 + kChunk - 1) / kChunk;
+    cs.nw = nchunks > warp ? (nchunks - warp + kWarps - 1) / kWarps : 0;  // this warp's chunks
+    cs.warp = warp;
+    cs.lane = lane;
+    cs.h = h;
+    cs.fast = (p.g.page_size % kChunk) == 0;
+    cs.pol = policy_evict_first();
+    cs.win = -1;
+    cs.mypage = -1;
+    return true;
+}
+
+__device__ __forceinline__ void init_bars(CtaRing& R, int warp, int lane) {
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < kStages; ++st) mbar_init(&R.bars[warp][st], 1);
+        fence_mbar_init();
+    }
+}
+
+// =====================================================================================
+// G = 8: heads on M, fp16 q.K
+// =====================================================================================
+template <int G>
+__global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p) {
+    __shared__ __align__(128) CtaRing R;
+    __shared__ uint32_t As[8 * 4 * 32];  // q.K A operand in fragment order: [k-step][reg][lane]
+    __shared__ float qsum_s[kMaxGroup];
+
+    const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2, pq = lane & 3;  // mma group id / thread in group
+    ChunkStream cs;
+    if (!begin_split(p, R, cs, warp, lane, tid)) return;
+    init_bars(R, warp, lane);
+    for (int w = tid; w < 8 * 4 * 32; w += kThreads) As[w] = 0u;
+    __syncthreads();
+    const int nw = cs.nw, t1 = cs.t1;
     const int pre = nw < kStages ? nw : kStages;
-    for (int i = 0; i < pre; ++i) issue(i, i);
+    for (int i = 0; i < pre; ++i) cs.issue(p, i, i);
 
     // ---------------- q' = q H_blk * log2(e)/sqrt(D) as fp16 hi/lo, fragment order ----------------
     for (int row = warp; row < G; row += kWarps) {
-        const uint2 raw = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.a.q) +
-                                                               (int64_t(s) * Hq + h * G + row) * kHeadDim) + lane);
-        float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
-                      __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};  // dims 4 lane + c
-        float sc = p.qscale;
-        if (p.g.mode == 2) {
-            const int b = p.g.bdr_block;
-            // strides 1 and 2 inside the lane, 4 .. 64 across lanes (lane bit = stride / 4)
-            float y0 = x[0] + x[1], y1 = x[0] - x[1], y2 = x[2] + x[3], y3 = x[2] - x[3];
-            x[0] = y0 + y2;
-            x[2] = y0 - y2;
-            x[1] = y1 + y3;
-            x[3] = y1 - y3;
-            for (int hs = 4; hs < b; hs <<= 1) {
-                const bool upper = (lane & (hs >> 2)) != 0;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float other = __shfl_xor_sync(0xffffffffu, x[c], hs >> 2);
-                    x[c] = upper ? other - x[c] : x[c] + other;
-                }
-            }
-            sc *= rsqrtf(float(b));
-        }
+        float x[4];
+        load_q_rotated(p, int64_t(s) * p.g.Hq + h * G + row, lane, x);
         float tsum = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            x[c] *= sc;
-            tsum += x[c];
-        }
+        for (int c = 0; c < 4; ++c) tsum += x[c];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, o);
+        for (int o = 16; o > 0; o >>= 1) tsum += __shfl_xor_sync(kFull, tsum, o);
         if (lane == 0) qsum_s[row] = tsum;
         uint16_t* A16 = reinterpret_cast<uint16_t*>(As);
 #pragma unroll
@@ -256,28 +387,26 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
     const float qsh = qsum_s[gq < G ? gq : 0];
 
     // ---------------- main loop over this warp's chunks ----------------
-    float m = -INFINITY, l = 0.0f, Z = 0.0f;  // softmax state of head gq (q.K layout)
-    float O[8][4];                            // P.V accumulators: dims x heads (2 pq, 2 pq + 1)
+    // softmax state of head gq (q.K layout); rows gq >= G stand for no head: their m stays 0
+    // and every score -inf, so they never trigger a rescale and their weights are 0
+    const bool gval = gq < G;
+    float m = gval ? -INFINITY : 0.0f, l = 0.0f, Z = 0.0f;
+    float O[8][4];  // P.V accumulators: dims x heads (2 pq, 2 pq + 1)
 #pragma unroll
     for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.0f;
     const int tokA = sigma(2 * pq), tokB = sigma(2 * pq + 1), tokK = sigma(gq);
 
     for (int i = 0; i < nw; ++i) {
         const int slot = i % kStages;
-        if (!mbar_wait(&bars[warp][slot], (i / kStages) & 1)) {
+        if (!mbar_wait(&R.bars[warp][slot], (i / kStages) & 1)) {
             flag_error(p.err, kErrTimeout);
             break;
         }
-        const uint8_t* st = ring[warp][slot];
-        const uint32_t vmask = smask[warp][slot];
-        const int tb = t0 + (warp + kWarps * i) * kChunk;
-        {  // each lane converts one (scale, zero) word: lanes 0..15 K, 16..31 V
-            const uint32_t w = reinterpret_cast<const uint32_t*>(st + kOffKs)[lane];
-            const float sc = half_lo(w), zr = half_hi(w);
-            // values use centred codes c - 8, so their offset is zero + 8 scale
-            szf[warp][lane >> 4][lane & 15] = make_float2(sc, lane < 16 ? zr : zr + 8.0f * sc);
-            __syncwarp();
-        }
+        const uint8_t* st = R.stage[warp][slot];
+        const uint32_t vmask = R.mask[warp][slot];
+        const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
+        // keys: the scale takes the 2^24 of the subnormal codes
+        stage_szf(R, st, warp, lane, kTwo24);
 
         // ---- scores: q' . codes for the two 8-token n-tiles ----
         float C[2][4];
@@ -293,33 +422,32 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
                 mma16816(C[tau], A[2 * wi + 1], ws & 0x000F000Fu, ws & 0x00F000F0u);
             }
         }
+        // A chunk whose 16 tokens all lie before the end and on valid pages needs no
+        // per-token masks (the common case).
+        const bool full = (tb + kChunk <= t1) && (vmask == 0xFFFFu);
         float sc[2][2];
-        int loc[2][2];
 #pragma unroll
-        for (int tau = 0; tau < 2; ++tau) {
+        for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int lt = 8 * tau + (e ? tokB : tokA);
-                loc[tau][e] = lt;
-                const float2 kz = szf[warp][0][lt];
-                const float S = (C[tau][e] + C[tau][2 + e]) * kTwo24;
-                const float v = kz.x * S + kz.y * qsh;
-                const bool valid = (gq < G) && (tb + lt < t1) && ((vmask >> lt) & 1u);
+                const float2 kz = R.szf[warp][0][lt];
+                const float v = fmaf(kz.x, C[tau][e] + C[tau][2 + e], kz.y * qsh);
+                const bool valid = gval && (full || ((tb + lt < t1) && ((vmask >> lt) & 1u)));
                 sc[tau][e] = valid ? v : -INFINITY;
             }
-        }
         // ---- online softmax (log2 domain) for head gq ----
         float cm = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
-        cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+        cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 1));
+        cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 2));
         const float mn = fmaxf(m, cm);
-        if (__any_sync(0xffffffffu, mn > m)) {
+        if (__any_sync(kFull, mn > m)) {
             const float alpha = (mn > m) ? fast_exp2(m - mn) : 1.0f;
             l *= alpha;
             Z *= alpha;
             m = mn;
-            const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * pq);
-            const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * pq + 4);
+            const float a0 = __shfl_sync(kFull, alpha, 8 * pq);
+            const float a1 = __shfl_sync(kFull, alpha, 8 * pq + 4);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 O[j][0] *= a0;
@@ -333,11 +461,19 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         for (int tau = 0; tau < 2; ++tau) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                // masked tokens (past the end, skipped pages, stale slots) may hold any bits in
-                // their scale/zero word: never let them reach an operand, even times 0
-                const bool live = sc[tau][e] != -INFINITY;
-                const float pr = live ? fast_exp2(sc[tau][e] - m) : 0.0f;
-                const float2 vz = live ? szf[warp][1][loc[tau][e]] : make_float2(0.0f, 0.0f);
+                const int lt = 8 * tau + (e ? tokB : tokA);
+                float pr;
+                float2 vz;
+                if (full) {  // rows past the group hold m = 0 and scores -inf: weight 0
+                    pr = fast_exp2(sc[tau][e] - m);
+                    vz = R.szf[warp][1][lt];
+                } else {
+                    // masked tokens (past the end, skipped pages, stale slots) may hold any bits
+                    // in their scale/zero word: never let them reach an operand, even times 0
+                    const bool live = sc[tau][e] != -INFINITY;
+                    pr = live ? fast_exp2(sc[tau][e] - m) : 0.0f;
+                    vz = live ? R.szf[warp][1][lt] : make_float2(0.0f, 0.0f);
+                }
                 l += pr;
                 Z += pr * vz.y;
                 pt_[tau][e] = pr * vz.x;
@@ -347,48 +483,21 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         const uint32_t b1 = pack_half2(pt_[1][0], pt_[1][1]);
         const uint32_t b0l = pack_half2(pt_[0][0] - half_lo(b0), pt_[0][1] - half_hi(b0));
         const uint32_t b1l = pack_half2(pt_[1][0] - half_lo(b1), pt_[1][1] - half_hi(b1));
-
-        // ---- P . V: A = codes of tokens (tokA, tokB), (8+tokA, 8+tokB), bytes [8 gq, 8 gq + 8) ----
-        const uint8_t* vc = st + kOffV + 8 * gq;
-        const uint2 v00 = *reinterpret_cast<const uint2*>(vc + tokA * 64);
-        const uint2 v01 = *reinterpret_cast<const uint2*>(vc + tokB * 64);
-        const uint2 v10 = *reinterpret_cast<const uint2*>(vc + (8 + tokA) * 64);
-        const uint2 v11 = *reinterpret_cast<const uint2*>(vc + (8 + tokB) * 64);
-#pragma unroll
-        for (int wq = 0; wq < 2; ++wq) {
-            const uint32_t x00 = wq ? v00.y : v00.x, x01 = wq ? v01.y : v01.x;
-            const uint32_t x10 = wq ? v10.y : v10.x, x11 = wq ? v11.y : v11.x;
-#pragma unroll
-            for (int bp = 0; bp < 2; ++bp) {
-                const uint32_t sel = bp ? 0x7632u : 0x5410u;
-                uint32_t P0 = prmt(x00, x01, sel), P1 = prmt(x10, x11, sel);
-#pragma unroll
-                for (int sh = 0; sh < 2; ++sh) {
-                    const int jv = 4 * wq + 2 * bp + sh;  // byte of the thread's 8-byte slice
-                    // centred codes (c - 8) 2^-24 and 16 (c - 8) 2^-24: exact subnormal fp16
-                    const uint32_t a[4] = {hadd2u(P0 & 0x000F000Fu, kMinus8), hadd2u(P0 & 0x00F000F0u, kMinus128),
-                                           hadd2u(P1 & 0x000F000Fu, kMinus8), hadd2u(P1 & 0x00F000F0u, kMinus128)};
-                    mma16816(O[jv], a, b0, b1);
-                    mma16816(O[jv], a, b0l, b1l);
-                    P0 >>= 8;
-                    P1 >>= 8;
-                }
-            }
-        }
+        pv_chunk<true>(O, st, gq, tokA, tokB, b0, b1, b0l, b1l);
         __syncwarp();
-        if (i + kStages < nw) issue(i + kStages, slot);
+        if (i + kStages < nw) cs.issue(p, i + kStages, slot);
     }
 
     // ---------------- per-head totals, undo the 2^-24 code scale, merge the warps ----------------
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    Z += __shfl_xor_sync(0xffffffffu, Z, 1);
-    Z += __shfl_xor_sync(0xffffffffu, Z, 2);
-    const float Z0 = __shfl_sync(0xffffffffu, Z, 8 * pq), Z1 = __shfl_sync(0xffffffffu, Z, 8 * pq + 4);
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    Z += __shfl_xor_sync(kFull, Z, 1);
+    Z += __shfl_xor_sync(kFull, Z, 2);
+    const float Z0 = __shfl_sync(kFull, Z, 8 * pq), Z1 = __shfl_sync(kFull, Z, 8 * pq + 4);
     __syncthreads();  // every ring is drained; reuse it for the merge
-    float* mo = reinterpret_cast<float*>(&ring[0][0][0]);  // [warp][G][128]
-    float* mm = mo + kWarps * G * kHeadDim;                // [warp][G]
-    float* ml = mm + kWarps * G;                           // [warp][G]
+    float* mo = reinterpret_cast<float*>(&R.stage[0][0][0]);  // [warp][G][128]
+    float* mm = mo + kWarps * G * kHeadDim;                   // [warp][G]
+    float* ml = mm + kWarps * G;                              // [warp][G]
     const int h0 = 2 * pq, h1 = 2 * pq + 1;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -407,23 +516,192 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         ml[warp * G + gq] = l;
     }
     __syncthreads();
+    store_partials<G>(p, mo, mm, ml, s, k, h, tid);
+}
+
+// =====================================================================================
+// G <= 4: tokens on M, int8 q.K
+// =====================================================================================
+template <int G>
+__global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p) {
+    static_assert(G >= 1 && G <= 4, "tokens-on-M tile serves up to 4 query heads per KV head");
+    __shared__ __align__(128) CtaRing R;
+    __shared__ uint32_t Bs[4 * 2 * 32];  // q.K B operand (4 x s8 per word) in fragment order: [k-step][reg][lane]
+    __shared__ float qsc_s[4], qsn_s[4];  // per head: fixed-point step of q', sum of the fixed-point q'
+
+    const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2, pq = lane & 3;
+    ChunkStream cs;
+    if (!begin_split(p, R, cs, warp, lane, tid)) return;
+    init_bars(R, warp, lane);
+    for (int w = tid; w < 4 * 2 * 32; w += kThreads) Bs[w] = 0u;
+    __syncthreads();
+    const int nw = cs.nw, t1 = cs.t1;
+    const int pre = nw < kStages ? nw : kStages;
+    for (int i = 0; i < pre; ++i) cs.issue(p, i, i);
+
+    // ---------------- q' as 16-bit fixed point per head, B fragment order ----------------
+    // k-step j, k-slot 4 pq + i (register 0) / 16 + 4 pq + i (register 1) stand for dim
+    // 32 pq + 8 j + 2 i (+ 1): the low / high nibbles of bytes 16 pq + 4 j + i.
+    // Column n = 2 head + part: part 0 holds hi, part 1 lo of q_int = 256 hi + lo.
+    for (int row = warp; row < G; row += kWarps) {
+        float x[4];
+        load_q_rotated(p, int64_t(s) * p.g.Hq + h * G + row, lane, x);
+        float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float M = -INFINITY;
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+        const float inv = amax > 0.0f ? float(kQFix) / amax : 0.0f;
+        int qi[4], isum = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mm[w * G + g]);
-        float acc = 0.0f, lt = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float mw = mm[w * G + g];
-            const float f = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - M);
-            acc += f * mo[(w * G + g) * kHeadDim + tid];
-            lt += f * ml[w * G + g];
+        for (int c = 0; c < 4; ++c) {
+            qi[c] = __float2int_rn(x[c] * inv);  // |qi| <= kQFix
+            isum += qi[c];
         }
-        const int64_t r = partial_row(p, s, k, h * G + g);
-        p.ws_o[r * kHeadDim + tid] = acc;
-        if (tid == 0) p.ws_ml[r] = make_float2(M, lt);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(kFull, isum, o);
+        if (lane == 0) {
+            qsc_s[row] = amax / float(kQFix);
+            qsn_s[row] = float(isum);
+        }
+        uint8_t* B8 = reinterpret_cast<uint8_t*>(Bs);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int d = 4 * lane + c;
+            const int dp = d >> 5, j = (d >> 3) & 3, i = (d >> 1) & 3, r = d & 1;
+            const int hi = (qi[c] + 128) >> 8, lo = qi[c] - 256 * hi;  // both in [-128, 127]
+            B8[((j * 2 + r) * 32 + 4 * (2 * row) + dp) * 4 + i] = uint8_t(hi);
+            B8[((j * 2 + r) * 32 + 4 * (2 * row + 1) + dp) * 4 + i] = uint8_t(lo);
+        }
     }
+    __syncthreads();
+    uint32_t Bq[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) Bq[j][r] = Bs[(j * 2 + r) * 32 + lane];
+
+    // ---------------- main loop over this warp's chunks ----------------
+    // Thread (gq, pq) scores tokens tk, tk + 8 against head pq; heads >= G hold m = 0 and
+    // scores -inf, so they never trigger a rescale and their weights are 0.
+    const bool hv = pq < G;
+    const float qsc = hv ? qsc_s[pq] : 0.0f, qsn = hv ? qsn_s[pq] : 0.0f;
+    float m = hv ? -INFINITY : 0.0f, l = 0.0f, Z = 0.0f;
+    float O[8][4];  // P.V accumulators: dims x (head pq high, head pq low)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.0f;
+    const int tk = sigma(gq), tokA = sigma(2 * pq), tokB = sigma(2 * pq + 1);
+    // P.V B column gq = (head gq >> 1, part gq & 1) wants tokens tokA, tokB (+ 8) of that head,
+    // which q.K left in lanes srcA = (row 2 pq, head) and srcB = (row 2 pq + 1, head).
+    // Even rows send their high words first, odd rows their low words, so each
+    // shuffle serves both parts.
+    const bool part = (gq & 1) != 0;
+    const int srcA = 4 * (2 * pq) + (gq >> 1), srcB = srcA + 4;
+    const int src1 = part ? srcB : srcA, src2 = part ? srcA : srcB;
+    const uint32_t sel0 = part ? 0x1054u : 0x5410u, sel1 = part ? 0x3276u : 0x7632u;
+
+    for (int i = 0; i < nw; ++i) {
+        const int slot = i % kStages;
+        if (!mbar_wait(&R.bars[warp][slot], (i / kStages) & 1)) {
+            flag_error(p.err, kErrTimeout);
+            break;
+        }
+        const uint8_t* st = R.stage[warp][slot];
+        const uint32_t vmask = R.mask[warp][slot];
+        const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
+        stage_szf(R, st, warp, lane, 1.0f);
+
+        // ---- scores: codes (tokens tk, tk + 8; bytes [16 pq, 16 pq + 16)) . q_int ----
+        const uint4 k0 = *reinterpret_cast<const uint4*>(st + tk * 64 + 16 * pq);
+        const uint4 k1 = *reinterpret_cast<const uint4*>(st + (tk + 8) * 64 + 16 * pq);
+        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+        int D[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t a[4] = {w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
+                                   (w1[j] >> 4) & 0x0F0F0F0Fu};
+            mma16832_u8s8(D, a, Bq[j][0], Bq[j][1]);
+        }
+        const float S0 = float(D[0] * 256 + D[1]), S1 = float(D[2] * 256 + D[3]);  // |S| < 2^26
+        const float2 kz0 = R.szf[warp][0][tk], kz1 = R.szf[warp][0][tk + 8];
+        const float v0 = qsc * fmaf(kz0.x, S0, kz0.y * qsn), v1 = qsc * fmaf(kz1.x, S1, kz1.y * qsn);
+        const bool full = (tb + kChunk <= t1) && (vmask == 0xFFFFu);
+        const bool ok0 = hv && (full || ((tb + tk < t1) && ((vmask >> tk) & 1u)));
+        const bool ok1 = hv && (full || ((tb + tk + 8 < t1) && ((vmask >> (tk + 8)) & 1u)));
+        const float sc0 = ok0 ? v0 : -INFINITY, sc1 = ok1 ? v1 : -INFINITY;
+
+        // ---- online softmax (log2 domain) for head pq: the 16 tokens sit in lanes pq + 4 n ----
+        float cm = fmaxf(sc0, sc1);
+        cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 4));
+        cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 8));
+        cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 16));
+        const float mn = fmaxf(m, cm);
+        if (__any_sync(kFull, mn > m)) {
+            const float alpha = (mn > m) ? fast_exp2(m - mn) : 1.0f;
+            l *= alpha;
+            Z *= alpha;
+            m = mn;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                O[j][0] *= alpha;
+                O[j][1] *= alpha;
+                O[j][2] *= alpha;
+                O[j][3] *= alpha;
+            }
+        }
+        float p0, p1;
+        float2 vz0, vz1;
+        if (full) {
+            p0 = fast_exp2(sc0 - m);
+            p1 = fast_exp2(sc1 - m);
+            vz0 = R.szf[warp][1][tk];
+            vz1 = R.szf[warp][1][tk + 8];
+        } else {
+            // masked tokens (past the end, skipped pages, stale slots) may hold any bits
+            // in their scale/zero word: never let them reach an operand, even times 0
+            const float2 zz = make_float2(0.0f, 0.0f);
+            p0 = ok0 ? fast_exp2(sc0 - m) : 0.0f;
+            p1 = ok1 ? fast_exp2(sc1 - m) : 0.0f;
+            vz0 = ok0 ? R.szf[warp][1][tk] : zz;
+            vz1 = ok1 ? R.szf[warp][1][tk + 8] : zz;
+        }
+        l += p0 + p1;
+        Z = fmaf(p0, vz0.y, fmaf(p1, vz1.y, Z));
+        const float P0 = p0 * vz0.x, P1 = p1 * vz1.x;
+        const uint32_t HI = pack_half2(P0, P1);
+        const uint32_t LO = pack_half2(P0 - half_lo(HI), P1 - half_hi(HI));
+        // ---- to the P.V B layout: (tokA, tokB) and (tokA + 8, tokB + 8) of column gq ----
+        const uint32_t R1 = __shfl_sync(kFull, part ? LO : HI, src1);
+        const uint32_t R2 = __shfl_sync(kFull, part ? HI : LO, src2);
+        pv_chunk<false>(O, st, gq, tokA, tokB, prmt(R1, R2, sel0), prmt(R1, R2, sel1), 0u, 0u);
+        __syncwarp();
+        if (i + kStages < nw) cs.issue(p, i + kStages, slot);
+    }
+
+    // ---------------- per-head totals, undo the 2^-24 code scale, merge the warps ----------------
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        l += __shfl_xor_sync(kFull, l, o);
+        Z += __shfl_xor_sync(kFull, Z, o);
+    }
+    __syncthreads();  // every ring is drained; reuse it for the merge
+    float* mo = reinterpret_cast<float*>(&R.stage[0][0][0]);  // [warp][G][128]
+    float* mm = mo + kWarps * G * kHeadDim;                   // [warp][G]
+    float* ml = mm + kWarps * G;                              // [warp][G]
+    if (hv) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int d = 16 * gq + 2 * j;
+            mo[(warp * G + pq) * kHeadDim + d] = (O[j][0] + O[j][1]) * kTwo24 + Z;
+            mo[(warp * G + pq) * kHeadDim + d + 1] = (O[j][2] + O[j][3]) * kTwo20 + Z;
+        }
+        if (gq == 0) {
+            mm[warp * G + pq] = m;
+            ml[warp * G + pq] = l;
+        }
+    }
+    __syncthreads();
+    store_partials<G>(p, mo, mm, ml, s, k, h, tid);
 }
 
 }  // namespace
@@ -431,9 +709,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s) {
     const dim3 grid(p.max_splits, p.g.H, p.a.batch);
     switch (p.g.Hq / p.g.H) {
-        case 1: decode_mma_kernel<1><<<grid, kThreads, 0, s>>>(p); break;
-        case 2: decode_mma_kernel<2><<<grid, kThreads, 0, s>>>(p); break;
-        case 4: decode_mma_kernel<4><<<grid, kThreads, 0, s>>>(p); break;
+        case 1: decode_tok_kernel<1><<<grid, kThreads, 0, s>>>(p); break;
+        case 2: decode_tok_kernel<2><<<grid, kThreads, 0, s>>>(p); break;
+        case 4: decode_tok_kernel<4><<<grid, kThreads, 0, s>>>(p); break;
         case 8: decode_mma_kernel<8><<<grid, kThreads, 0, s>>>(p); break;
         default: return cudaErrorInvalidValue;
     }
