@@ -12,11 +12,11 @@
 // chunks of its split (round robin), with its own online-softmax state.  The
 // CTA issues its first copies before anything else, then prepares q, so the
 // prologue hides under the first memory latency.
-//   * Staging: per warp a ring of 4 shared-memory stages; one lane issues 1-D
-//     bulk async copies (cp.async.bulk, no multicast) of the chunk's K codes,
-//     V codes and scale/zero words (2176 B) on an mbarrier; every wait is
-//     bounded.  Page sizes that are not a multiple of 16 take a per-token
-//     gather instead.
+//   * Staging: per warp a ring of 4 shared-memory stages, 4 chunks in flight;
+//     all 32 lanes copy a chunk's K codes, V codes and scale/zero words (2176
+//     B) with 16-byte cp.async (one copy group per chunk), so no lane runs a
+//     divergent issue path.  Page sizes that are not a multiple of 16 take a
+//     per-token gather of the same form.
 //   * P.V (both tiles): D[16 dims x 8 cols] += A[16 dims x 16 tokens] B[16 tokens
 //     x 8 cols].  A = V codes of two tokens per register (PRMT + AND) masked
 //     into fp16 lanes, where a nibble c is the exact subnormal c 2^-24, and
@@ -88,12 +88,20 @@ __device__ __forceinline__ void mma16832_u8s8(int (&c)[4], const uint32_t (&a)[4
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
-            "r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-        : "memory");
+// 16-byte asynchronous global -> shared copy (L2 only), completed by the copy-group waits below
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// this thread's copy groups, all but the n most recent, have landed
+template <int n>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -120,7 +128,6 @@ __device__ __forceinline__ int sigma(int n) { return n ^ ((n >> 2) & 1); }
 // What a CTA keeps in shared memory for its warps' chunk streams.
 struct CtaRing {
     uint8_t stage[kWarps][kStages][kStageBytes];
-    uint64_t bars[kWarps][kStages];
     uint32_t mask[kWarps][kStages];     // tokens of the staged chunk on valid pages (bit per token)
     float2 szf[kWarps][2][kChunk];      // (scale, offset) of the current chunk: [warp][K / V][token]
 };
@@ -144,35 +151,40 @@ struct ChunkStream {
         return __shfl_sync(kFull, mypage, iw & 31);
     }
 
+    // Copies of chunk iw into ring slot by all 32 lanes (16-byte cp.async, no divergent
+    // issuer), then one commit: the stream always holds one copy group per chunk slot.
     __device__ __forceinline__ void issue(const DecodeParams& p, int iw, int slot) {
         uint8_t* st = r->stage[warp][slot];
-        uint64_t* bar = &r->bars[warp][slot];
         const int tb = t0 + (warp + kWarps * iw) * kChunk;
         const uint8_t* kpool = static_cast<const uint8_t*>(p.g.k_pool);
         const uint8_t* vpool = static_cast<const uint8_t*>(p.g.v_pool);
         const int H = p.g.H, ps = p.g.page_size;
         if (fast) {
+            // 16 consecutive slots of one page: 1 KiB of K codes, 1 KiB of V codes, 64 B of
+            // scale/zero words each; lane L copies bytes 16 L and 512 + 16 L of both code
+            // blocks, lanes 0..3 / 4..7 the K / V scale/zero words
             const int page = page_of(p, iw);
-            if (lane == 0) {
-                if (page >= 0 && page < p.g.num_pages) {
-                    const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, tb);
-                    r->mask[warp][slot] = 0xFFFFu;
-                    fence_proxy_async();
-                    mbar_expect_tx(bar, kStageBytes);
-                    bulk_g2s(st, kpool + row * 64, kCodeBytes, bar, pol);
-                    bulk_g2s(st + kOffV, vpool + row * 64, kCodeBytes, bar, pol);
-                    bulk_g2s(st + kOffKs, p.g.k_sz + row, kChunk * 4, bar, pol);
-                    bulk_g2s(st + kOffVs, p.g.v_sz + row, kChunk * 4, bar, pol);
-                } else {
-                    r->mask[warp][slot] = 0u;
-                    flag_error(p.err, kErrOOB);
+            const bool ok = page >= 0 && page < p.g.num_pages;
+            if (ok) {
+                const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, tb);
+                const uint8_t* kc = kpool + row * 64 + 16 * lane;
+                const uint8_t* vc = vpool + row * 64 + 16 * lane;
+                cp_async16(st + 16 * lane, kc, pol);
+                cp_async16(st + 512 + 16 * lane, kc + 512, pol);
+                cp_async16(st + kOffV + 16 * lane, vc, pol);
+                cp_async16(st + kOffV + 512 + 16 * lane, vc + 512, pol);
+                if (lane < 8) {
+                    const uint32_t* sz = (lane < 4 ? p.g.k_sz : p.g.v_sz) + row + 4 * (lane & 3);
+                    cp_async16(st + kOffKs + 16 * lane, sz, pol);  // V words follow the K words
                 }
-                mbar_arrive(bar);
+            } else if (lane == 0) {
+                flag_error(p.err, kErrOOB);
             }
+            if (lane == 0) r->mask[warp][slot] = ok ? 0xFFFFu : 0u;
         } else {
-            // gather: lanes 0..15 fetch K rows, lanes 16..31 V rows of tokens tb + (lane & 15)
-            const int i = lane & 15;
-            const bool isv = lane >= 16;
+            // gather: lane L copies half L & 1 of token tb + (L >> 1)'s K and V code rows and
+            // its K (even L) or V (odd L) scale/zero word
+            const int i = lane >> 1, hf = lane & 1;
             const int t = tb + i;
             bool ok = false;
             if (t < t1) {
@@ -180,22 +192,25 @@ struct ChunkStream {
                 ok = page >= 0 && page < p.g.num_pages;
                 if (ok) {
                     const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, t);
-                    const uint4* src = reinterpret_cast<const uint4*>((isv ? vpool : kpool) + row * 64);
-                    uint4* dst = reinterpret_cast<uint4*>(st + (isv ? kOffV : 0) + i * 64);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) dst[q4] = __ldg(src + q4);
-                    reinterpret_cast<uint32_t*>(st + (isv ? kOffVs : kOffKs))[i] =
-                        __ldg((isv ? p.g.v_sz : p.g.k_sz) + row);
-                } else if (!isv) {
+                    const int off = i * 64 + 32 * hf;
+                    const uint8_t* kc = kpool + row * 64 + 32 * hf;
+                    const uint8_t* vc = vpool + row * 64 + 32 * hf;
+                    cp_async16(st + off, kc, pol);
+                    cp_async16(st + off + 16, kc + 16, pol);
+                    cp_async16(st + kOffV + off, vc, pol);
+                    cp_async16(st + kOffV + off + 16, vc + 16, pol);
+                    cp_async4(st + (hf ? kOffVs : kOffKs) + 4 * i, (hf ? p.g.v_sz : p.g.k_sz) + row);
+                } else if (hf == 0) {
                     flag_error(p.err, kErrOOB);
                 }
             }
-            const uint32_t m = __ballot_sync(kFull, ok) & 0xFFFFu;
-            __syncwarp();
-            if (lane == 0) {
-                r->mask[warp][slot] = m;
-                mbar_arrive(bar);
-            }
+            uint32_t m = __ballot_sync(kFull, ok);
+            m = (m & 0x55555555u);  // one bit per token (even lanes) -> compact to bit i
+            m = (m | (m >> 1)) & 0x33333333u;
+            m = (m | (m >> 2)) & 0x0F0F0F0Fu;
+            m = (m | (m >> 4)) & 0x00FF00FFu;
+            m = (m | (m >> 8)) & 0x0000FFFFu;
+            if (lane == 0) r->mask[warp][slot] = m;
         }
     }
 };
@@ -324,14 +339,6 @@ __device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, C
     return true;
 }
 
-__device__ __forceinline__ void init_bars(CtaRing& R, int warp, int lane) {
-    if (lane == 0) {
-#pragma unroll
-        for (int st = 0; st < kStages; ++st) mbar_init(&R.bars[warp][st], 1);
-        fence_mbar_init();
-    }
-}
-
 // =====================================================================================
 // G = 8: heads on M, fp16 q.K
 // =====================================================================================
@@ -346,12 +353,13 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
     const int gq = lane >> 2, pq = lane & 3;  // mma group id / thread in group
     ChunkStream cs;
     if (!begin_split(p, R, cs, warp, lane, tid)) return;
-    init_bars(R, warp, lane);
     for (int w = tid; w < 8 * 4 * 32; w += kThreads) As[w] = 0u;
     __syncthreads();
     const int nw = cs.nw, t1 = cs.t1;
-    const int pre = nw < kStages ? nw : kStages;
-    for (int i = 0; i < pre; ++i) cs.issue(p, i, i);
+    for (int i = 0; i < kStages; ++i) {
+        if (i < nw) cs.issue(p, i, i);
+        cp_async_commit();
+    }
 
     // ---------------- q' = q H_blk * log2(e)/sqrt(D) as fp16 hi/lo, fragment order ----------------
     for (int row = warp; row < G; row += kWarps) {
@@ -398,10 +406,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
 
     for (int i = 0; i < nw; ++i) {
         const int slot = i % kStages;
-        if (!mbar_wait(&R.bars[warp][slot], (i / kStages) & 1)) {
-            flag_error(p.err, kErrTimeout);
-            break;
-        }
+        cp_async_wait<kStages - 1>();  // chunk i's group (the stream keeps kStages groups)
+        __syncwarp();                   // ... and every lane's copies of it
         const uint8_t* st = R.stage[warp][slot];
         const uint32_t vmask = R.mask[warp][slot];
         const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
@@ -484,8 +490,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         const uint32_t b0l = pack_half2(pt_[0][0] - half_lo(b0), pt_[0][1] - half_hi(b0));
         const uint32_t b1l = pack_half2(pt_[1][0] - half_lo(b1), pt_[1][1] - half_hi(b1));
         pv_chunk<true>(O, st, gq, tokA, tokB, b0, b1, b0l, b1l);
-        __syncwarp();
+        __syncwarp();  // every lane is done with this slot
         if (i + kStages < nw) cs.issue(p, i + kStages, slot);
+        cp_async_commit();
     }
 
     // ---------------- per-head totals, undo the 2^-24 code scale, merge the warps ----------------
@@ -534,12 +541,13 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
     const int gq = lane >> 2, pq = lane & 3;
     ChunkStream cs;
     if (!begin_split(p, R, cs, warp, lane, tid)) return;
-    init_bars(R, warp, lane);
     for (int w = tid; w < 4 * 2 * 32; w += kThreads) Bs[w] = 0u;
     __syncthreads();
     const int nw = cs.nw, t1 = cs.t1;
-    const int pre = nw < kStages ? nw : kStages;
-    for (int i = 0; i < pre; ++i) cs.issue(p, i, i);
+    for (int i = 0; i < kStages; ++i) {
+        if (i < nw) cs.issue(p, i, i);
+        cp_async_commit();
+    }
 
     // ---------------- q' as 16-bit fixed point per head, B fragment order ----------------
     // k-step j, k-slot 4 pq + i (register 0) / 16 + 4 pq + i (register 1) stand for dim
@@ -602,10 +610,8 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
 
     for (int i = 0; i < nw; ++i) {
         const int slot = i % kStages;
-        if (!mbar_wait(&R.bars[warp][slot], (i / kStages) & 1)) {
-            flag_error(p.err, kErrTimeout);
-            break;
-        }
+        cp_async_wait<kStages - 1>();  // chunk i's group (the stream keeps kStages groups)
+        __syncwarp();                   // ... and every lane's copies of it
         const uint8_t* st = R.stage[warp][slot];
         const uint32_t vmask = R.mask[warp][slot];
         const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
@@ -674,8 +680,9 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         const uint32_t R1 = __shfl_sync(kFull, part ? LO : HI, src1);
         const uint32_t R2 = __shfl_sync(kFull, part ? HI : LO, src2);
         pv_chunk<false>(O, st, gq, tokA, tokB, prmt(R1, R2, sel0), prmt(R1, R2, sel1), 0u, 0u);
-        __syncwarp();
+        __syncwarp();  // every lane is done with this slot
         if (i + kStages < nw) cs.issue(p, i + kStages, slot);
+        cp_async_commit();
     }
 
     // ---------------- per-head totals, undo the 2^-24 code scale, merge the warps ----------------
