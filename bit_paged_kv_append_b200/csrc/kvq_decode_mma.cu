@@ -79,6 +79,15 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D[16 x 8] += A[16 x 32] (s8) B[32 x 8] (u8), int32 accumulation
+__device__ __forceinline__ void mma16832_s8u8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // D[16 x 8] += A[16 x 32] (u8) B[32 x 8] (s8), int32 accumulation
 __device__ __forceinline__ void mma16832_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -343,17 +352,17 @@ __device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, C
 // G = 8: heads on M, fp16 q.K
 // =====================================================================================
 template <int G>
-__global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p) {
     __shared__ __align__(128) CtaRing R;
-    __shared__ uint32_t As[8 * 4 * 32];  // q.K A operand in fragment order: [k-step][reg][lane]
-    __shared__ float qsum_s[kMaxGroup];
+    __shared__ uint32_t As[4 * 4 * 32];  // q.K A operand (4 x s8 per word) in fragment order: [k-step][reg][lane]
+    __shared__ float qsc_s[kMaxGroup], qsn_s[kMaxGroup];  // per head: fixed-point step, sum of q_int
 
     const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, pq = lane & 3;  // mma group id / thread in group
     ChunkStream cs;
     if (!begin_split(p, R, cs, warp, lane, tid)) return;
-    for (int w = tid; w < 8 * 4 * 32; w += kThreads) As[w] = 0u;
+    for (int w = tid; w < 4 * 4 * 32; w += kThreads) As[w] = 0u;
     __syncthreads();
     const int nw = cs.nw, t1 = cs.t1;
     for (int i = 0; i < kStages; ++i) {
@@ -361,38 +370,46 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         cp_async_commit();
     }
 
-    // ---------------- q' = q H_blk * log2(e)/sqrt(D) as fp16 hi/lo, fragment order ----------------
+    // ---------------- q' as 16-bit fixed point per head, A fragment order ----------------
+    // k-step j, k-slot 4 pq + i (registers 0, 1) / 16 + 4 pq + i (registers 2, 3) stand for
+    // dim 32 pq + 8 j + 2 i (+ 1); rows 0..7 hold hi, rows 8..15 lo of q_int = 256 hi + lo.
     for (int row = warp; row < G; row += kWarps) {
         float x[4];
         load_q_rotated(p, int64_t(s) * p.g.Hq + h * G + row, lane, x);
-        float tsum = 0.0f;
+        float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tsum += x[c];
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+        const float inv = amax > 0.0f ? float(kQFix) / amax : 0.0f;
+        int qi[4], isum = 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tsum += __shfl_xor_sync(kFull, tsum, o);
-        if (lane == 0) qsum_s[row] = tsum;
-        uint16_t* A16 = reinterpret_cast<uint16_t*>(As);
+        for (int c = 0; c < 4; ++c) {
+            qi[c] = __float2int_rn(x[c] * inv);  // |qi| <= kQFix
+            isum += qi[c];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(kFull, isum, o);
+        if (lane == 0) {
+            qsc_s[row] = amax / float(kQFix);
+            qsn_s[row] = float(isum);
+        }
+        uint8_t* A8 = reinterpret_cast<uint8_t*>(As);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int d = 4 * lane + c;
-            const float v = x[c] * ((d & 1) ? 0.0625f : 1.0f);  // odd d pairs with a high nibble (x16)
-            const __half hi = __float2half_rn(v);
-            const __half lo = __float2half_rn(v - __half2float(hi));
-            // inverse of dpos: d = 32 pp + 8 i + off
-            const int pp = d >> 5, i = (d >> 3) & 3, off = d & 7;
-            const int j = 2 * i + ((off >> 1) & 1), h8 = off & 1, e = off >> 2;
-            const int base = (j * 4 + 2 * h8) * 32 + 4 * row + pp;  // hi part: register 2 h8; lo part: + 1
-            A16[2 * base + e] = __half_as_ushort(hi);
-            A16[2 * (base + 32) + e] = __half_as_ushort(lo);
+            const int dp = d >> 5, j = (d >> 3) & 3, i = (d >> 1) & 3, odd = d & 1;
+            const int hi = (qi[c] + 128) >> 8, lo = qi[c] - 256 * hi;  // both in [-128, 127]
+            const int lw = 4 * row + dp;                                // lane of row gq = row
+            A8[((j * 4 + 2 * odd) * 32 + lw) * 4 + i] = uint8_t(hi);
+            A8[((j * 4 + 2 * odd + 1) * 32 + lw) * 4 + i] = uint8_t(lo);
         }
     }
     __syncthreads();
-    uint32_t A[8][4];
+    uint32_t A[4][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int r = 0; r < 4; ++r) A[j][r] = As[(j * 4 + r) * 32 + lane];
-    const float qsh = qsum_s[gq < G ? gq : 0];
+    const float qsc = gq < G ? qsc_s[gq] : 0.0f, qsn = gq < G ? qsn_s[gq] : 0.0f;
 
     // ---------------- main loop over this warp's chunks ----------------
     // softmax state of head gq (q.K layout); rows gq >= G stand for no head: their m stays 0
@@ -411,22 +428,19 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         const uint8_t* st = R.stage[warp][slot];
         const uint32_t vmask = R.mask[warp][slot];
         const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
-        // keys: the scale takes the 2^24 of the subnormal codes
-        stage_szf(R, st, warp, lane, kTwo24);
+        stage_szf(R, st, warp, lane, 1.0f);
 
-        // ---- scores: q' . codes for the two 8-token n-tiles ----
-        float C[2][4];
+        // ---- scores: q_int . codes for the two 8-token n-tiles (column gq: token 8 tau + tokK) ----
+        float C[2][2];
 #pragma unroll
         for (int tau = 0; tau < 2; ++tau) {
             const uint4 kw = *reinterpret_cast<const uint4*>(st + (8 * tau + tokK) * 64 + 16 * pq);
             const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
-            C[tau][0] = C[tau][1] = C[tau][2] = C[tau][3] = 0.0f;
+            int D[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-                const uint32_t ws = w[wi] >> 8;
-                mma16816(C[tau], A[2 * wi], w[wi] & 0x000F000Fu, w[wi] & 0x00F000F0u);
-                mma16816(C[tau], A[2 * wi + 1], ws & 0x000F000Fu, ws & 0x00F000F0u);
-            }
+            for (int j = 0; j < 4; ++j) mma16832_s8u8(D, A[j], w[j] & 0x0F0F0F0Fu, (w[j] >> 4) & 0x0F0F0F0Fu);
+            C[tau][0] = float(D[0] * 256 + D[2]);  // head gq, column 2 pq; |S| < 2^26
+            C[tau][1] = float(D[1] * 256 + D[3]);  // head gq, column 2 pq + 1
         }
         // A chunk whose 16 tokens all lie before the end and on valid pages needs no
         // per-token masks (the common case).
@@ -438,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
             for (int e = 0; e < 2; ++e) {
                 const int lt = 8 * tau + (e ? tokB : tokA);
                 const float2 kz = R.szf[warp][0][lt];
-                const float v = fmaf(kz.x, C[tau][e] + C[tau][2 + e], kz.y * qsh);
+                const float v = qsc * fmaf(kz.x, C[tau][e], kz.y * qsn);
                 const bool valid = gval && (full || ((tb + lt < t1) && ((vmask >> lt) & 1u)));
                 sc[tau][e] = valid ? v : -INFINITY;
             }
