@@ -239,6 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbar_init();
     }
     __syncthreads();
+    grid_dep_wait();  // inputs and cache as the previous grid left them
+    grid_dep_launch();
 
     if (warp == kRows / 32) {
         // ---------------- producer warp ----------------
@@ -383,8 +385,7 @@ cudaError_t launch_t(const CUtensorMap& km, const CUtensorMap& vm, const Params&
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    kern<<<grid, kThreads, kSmemBytes, s>>>(km, vm, p);
-    return cudaGetLastError();
+    return launch_overlapped(kern, dim3(grid), dim3(kThreads), kSmemBytes, s, km, vm, p);
 }
 
 }  // namespace

@@ -68,7 +68,11 @@ __global__ void __launch_bounds__(kThreads) bf16_split_kernel(Params p) {
     const int L = decode_len(p, s);
     if (k == 0 && h == 0 && tid == 0 && L != __ldg(p.a.seq_lens + s)) flag_error(p.err, kErrOOB);
     const int t0 = k * p.item_tokens;
-    if (t0 >= L) return;  // past the end of the sequence
+    if (t0 >= L) {  // past the end of the sequence
+        grid_dep_wait();  // still: no grid here completes before the one it follows
+        grid_dep_launch();
+        return;
+    }
     const int t1 = min(L, t0 + p.item_tokens);
     const int64_t out_row0 = partial_row(p, s, k, h * G);
 
@@ -86,6 +90,8 @@ __global__ void __launch_bounds__(kThreads) bf16_split_kernel(Params p) {
         for (int e = 0; e < 4; ++e) o[g][e] = 0.0f;
     }
     const int32_t* pt = p.a.page_table + int64_t(s) * p.a.pt_stride;
+    grid_dep_wait();  // the cache as the previous grid (an append) left it
+    grid_dep_launch();
 
     for (int base = t0 + 32 * warp; base < t1; base += 32 * kWarps) {
         const int t = base + lane;
@@ -211,6 +217,8 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Params p, int rotate_ou
     const int Hq = p.g.Hq;
     const int s = row / Hq, j = row % Hq;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    grid_dep_wait();  // the split kernel's partials
+    grid_dep_launch();
     const int n = (decode_len(p, s) + p.item_tokens - 1) / p.item_tokens;
     const int64_t stride = int64_t(Hq) * kHeadDim;  // next split, same query head
     float acc = 0.0f, l = 0.0f, M = -INFINITY;
@@ -270,14 +278,13 @@ cudaError_t launch_group(const Params& p, cudaStream_t st) {
     const int B = p.a.batch, H = p.g.H;
     cudaError_t e;
     if (p.g.mode == 0) {
-        bf16_split_kernel<G><<<dim3(p.max_splits, H, B), kThreads, 0, st>>>(p);
-        e = cudaGetLastError();
+        e = launch_overlapped(bf16_split_kernel<G>, dim3(p.max_splits, H, B), dim3(kThreads), 0, st, p);
     } else {
         e = launch_decode_mma(p, st);
     }
     if (e != cudaSuccess) return e;
-    merge_kernel<<<B * p.g.Hq, kThreads, 0, st>>>(p, p.g.mode == 2 && p.g.rotate_v);
-    return cudaGetLastError();
+    return launch_overlapped(merge_kernel, dim3(B * p.g.Hq), dim3(kThreads), 0, st, p,
+                             int(p.g.mode == 2 && p.g.rotate_v));
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -285,17 +292,18 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
 DecodePlan plan_decode(const CacheGeom& g, int batch, int max_seq_len, int num_sms) {
-    // Splits of a multiple of 64 tokens (4 warps x 16-token chunks), between 256 and 8192
-    // tokens (bounding how many steps one warp accumulates), sized so that a full batch at the length bound gives about 2.5 waves of
-    // resident split CTAs (4 per SM): long enough to amortise a CTA's start-up and merge,
-    // short enough to balance the tail.
+    // Splits of a multiple of 64 tokens (4 warps x 16-token chunks), between 512 and 4096
+    // tokens, sized so that a full batch at the length bound gives about 2.75 waves of
+    // resident split CTAs (5 per SM).  Measured on B200 over batch sizes 1..256 and
+    // lengths 2k..1M: shorter splits pay their start-up and merge more often, longer ones
+    // leave a tail; 4096 also bounds how many steps one warp accumulates.
     DecodePlan pl;
     const int64_t L = max_seq_len > 0 ? max_seq_len : 1;
-    const int64_t slots = int64_t(num_sms > 0 ? num_sms : 148) * 4;
-    int64_t it = (int64_t(batch) * g.H * L * 2 + 5 * slots - 1) / (5 * slots);
+    const int64_t slots = int64_t(num_sms > 0 ? num_sms : 148) * 5;
+    int64_t it = (int64_t(batch) * g.H * L * 4 + 11 * slots - 1) / (11 * slots);
     it = ((it + 63) / 64) * 64;
-    if (it < 256) it = 256;
-    if (it > 8192) it = 8192;
+    if (it < 512) it = 512;
+    if (it > 4096) it = 4096;
     pl.item_tokens = int(it);
     pl.max_splits = int((L + it - 1) / it);
     pl.max_items = batch * pl.max_splits;

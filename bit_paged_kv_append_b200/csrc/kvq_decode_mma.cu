@@ -10,8 +10,9 @@
 //
 // One CTA = (split, KV head, sequence), 4 warps; each warp walks 16-token
 // chunks of its split (round robin), with its own online-softmax state.  The
-// CTA issues its first copies before anything else, then prepares q, so the
-// prologue hides under the first memory latency.
+// CTA prepares q first (it may overlap the end of the previous grid in the
+// stream: programmatic dependent launch), then waits for that grid and starts
+// its copies.
 //   * Staging: per warp a ring of 4 shared-memory stages, 4 chunks in flight;
 //     all 32 lanes copy a chunk's K codes, V codes and scale/zero words (2176
 //     B) with 16-byte cp.async (one copy group per chunk), so no lane runs a
@@ -331,7 +332,11 @@ __device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, C
     const int L = decode_len(p, s);
     if (k == 0 && h == 0 && tid == 0 && L != __ldg(p.a.seq_lens + s)) flag_error(p.err, kErrOOB);
     const int t0 = k * p.item_tokens;
-    if (t0 >= L) return false;  // past the end of the sequence: no partial (the merge reads only real splits)
+    if (t0 >= L) {  // past the end of the sequence: no partial (the merge reads only real splits)
+        grid_dep_wait();  // still: no grid here completes before the one it follows
+        grid_dep_launch();
+        return false;
+    }
     cs.r = &R;
     cs.pt = p.a.page_table + int64_t(s) * p.a.pt_stride;
     cs.t0 = t0;
@@ -365,10 +370,6 @@ __global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p)
     for (int w = tid; w < 4 * 4 * 32; w += kThreads) As[w] = 0u;
     __syncthreads();
     const int nw = cs.nw, t1 = cs.t1;
-    for (int i = 0; i < kStages; ++i) {
-        if (i < nw) cs.issue(p, i, i);
-        cp_async_commit();
-    }
 
     // ---------------- q' as 16-bit fixed point per head, A fragment order ----------------
     // k-step j, k-slot 4 pq + i (registers 0, 1) / 16 + 4 pq + i (registers 2, 3) stand for
@@ -402,6 +403,13 @@ __global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p)
             A8[((j * 4 + 2 * odd) * 32 + lw) * 4 + i] = uint8_t(hi);
             A8[((j * 4 + 2 * odd + 1) * 32 + lw) * 4 + i] = uint8_t(lo);
         }
+    }
+    // q only (never written by an append) so far; the cache after the previous grid
+    grid_dep_wait();
+    grid_dep_launch();
+    for (int i = 0; i < kStages; ++i) {
+        if (i < nw) cs.issue(p, i, i);
+        cp_async_commit();
     }
     __syncthreads();
     uint32_t A[4][4];
@@ -558,10 +566,6 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
     for (int w = tid; w < 4 * 2 * 32; w += kThreads) Bs[w] = 0u;
     __syncthreads();
     const int nw = cs.nw, t1 = cs.t1;
-    for (int i = 0; i < kStages; ++i) {
-        if (i < nw) cs.issue(p, i, i);
-        cp_async_commit();
-    }
 
     // ---------------- q' as 16-bit fixed point per head, B fragment order ----------------
     // k-step j, k-slot 4 pq + i (register 0) / 16 + 4 pq + i (register 1) stand for dim
@@ -595,6 +599,13 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
             B8[((j * 2 + r) * 32 + 4 * (2 * row) + dp) * 4 + i] = uint8_t(hi);
             B8[((j * 2 + r) * 32 + 4 * (2 * row + 1) + dp) * 4 + i] = uint8_t(lo);
         }
+    }
+    // q only (never written by an append) so far; the cache after the previous grid
+    grid_dep_wait();
+    grid_dep_launch();
+    for (int i = 0; i < kStages; ++i) {
+        if (i < nw) cs.issue(p, i, i);
+        cp_async_commit();
     }
     __syncthreads();
     uint32_t Bq[4][2];
@@ -730,13 +741,12 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s) {
     const dim3 grid(p.max_splits, p.g.H, p.a.batch);
     switch (p.g.Hq / p.g.H) {
-        case 1: decode_tok_kernel<1><<<grid, kThreads, 0, s>>>(p); break;
-        case 2: decode_tok_kernel<2><<<grid, kThreads, 0, s>>>(p); break;
-        case 4: decode_tok_kernel<4><<<grid, kThreads, 0, s>>>(p); break;
-        case 8: decode_mma_kernel<8><<<grid, kThreads, 0, s>>>(p); break;
+        case 1: return launch_overlapped(decode_tok_kernel<1>, grid, dim3(kThreads), 0, s, p);
+        case 2: return launch_overlapped(decode_tok_kernel<2>, grid, dim3(kThreads), 0, s, p);
+        case 4: return launch_overlapped(decode_tok_kernel<4>, grid, dim3(kThreads), 0, s, p);
+        case 8: return launch_overlapped(decode_mma_kernel<8>, grid, dim3(kThreads), 0, s, p);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace kvq
