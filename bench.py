@@ -53,8 +53,9 @@ HEADLINE = {"batch16": ("bdr128_k", kvq.KV_INT4_BDR, 128, False),
             "decode64x8k": ("bdr128_k", kvq.KV_INT4_BDR, 128, False),
             "mixed256": ("bdr128_kv", kvq.KV_INT4_BDR, 128, True),
             "long1m": ("bdr128_k", kvq.KV_INT4_BDR, 128, False)}
+_DECODE_SOURCES = ["kvq_decode_mma.cu", "kvq_decode.cuh", "kvq_common.cuh", "kvq_internal.h"]
 KERNEL_SOURCES = {"append_kernel": ["kvq_append.cu", "kvq_common.cuh", "kvq_internal.h"],
-                  "decode_mma_kernel": ["kvq_decode_mma.cu", "kvq_decode.cuh", "kvq_common.cuh", "kvq_internal.h"]}
+                  "decode_tok_kernel": _DECODE_SOURCES, "decode_mma_kernel": _DECODE_SOURCES}
 
 
 def peak_hbm():
@@ -451,7 +452,10 @@ def main():
     dec_gbs = dec_b / (res["decode_ms"] / 1e3) / 1e9
     dominant = "append" if res["append_ms"] >= res["decode_ms"] else "decode"
     dom_gbs = app_gbs if dominant == "append" else dec_gbs
-    traffic = profiled_traffic("append_kernel" if dominant == "append" else "decode_mma_kernel", args.workload)
+    # the INT4 decode runs the tokens-on-M tile for up to 4 query heads per KV head, else heads-on-M
+    dec_kernel = "decode_tok_kernel" if w.Hq // w.H <= 4 else "decode_mma_kernel"
+    dom_kernel = "append_kernel" if dominant == "append" else dec_kernel
+    traffic = profiled_traffic(dom_kernel, args.workload)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -471,7 +475,7 @@ def main():
             "decode": {"us": res["decode_ms"] * 1e3, "algorithmic_bytes": dec_b, "gbs": dec_gbs,
                        "frac_of_peak": dec_gbs / peak, "frac_of_8tbs": dec_gbs / NOMINAL_HBM_GBS,
                        "note": "split + merge kernels"}},
-        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
+        "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
                      "frac": dom_gbs / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                      "traffic": traffic},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

@@ -135,6 +135,12 @@ __device__ __forceinline__ float half_hi(uint32_t w) { return __half2float(__ush
 // P.V load touches then fall on both 64-byte halves of the bank space.
 __device__ __forceinline__ int sigma(int n) { return n ^ ((n >> 2) & 1); }
 
+// Byte offset of byte b of V-code row r in a stage: rows with bit 1 set swap their
+// 32-byte halves, so the four rows (two even, two odd, one of each pair with bit 1
+// set) that one 8-byte P.V load reads in each half-warp hit four distinct 32-byte
+// bank groups.
+__device__ __forceinline__ int vrow_off(int r, int b) { return kOffV + 64 * r + (b ^ ((r & 2) << 4)); }
+
 // What a CTA keeps in shared memory for its warps' chunk streams.
 struct CtaRing {
     uint8_t stage[kWarps][kStages][kStageBytes];
@@ -179,10 +185,11 @@ struct ChunkStream {
                 const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, tb);
                 const uint8_t* kc = kpool + row * 64 + 16 * lane;
                 const uint8_t* vc = vpool + row * 64 + 16 * lane;
+                const int vu = 16 * (lane ^ ((lane >> 2) & 2));  // V rows swizzled (vrow_off)
                 cp_async16(st + 16 * lane, kc, pol);
                 cp_async16(st + 512 + 16 * lane, kc + 512, pol);
-                cp_async16(st + kOffV + 16 * lane, vc, pol);
-                cp_async16(st + kOffV + 512 + 16 * lane, vc + 512, pol);
+                cp_async16(st + kOffV + vu, vc, pol);
+                cp_async16(st + kOffV + 512 + vu, vc + 512, pol);
                 if (lane < 8) {
                     const uint32_t* sz = (lane < 4 ? p.g.k_sz : p.g.v_sz) + row + 4 * (lane & 3);
                     cp_async16(st + kOffKs + 16 * lane, sz, pol);  // V words follow the K words
@@ -203,12 +210,13 @@ struct ChunkStream {
                 if (ok) {
                     const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, t);
                     const int off = i * 64 + 32 * hf;
+                    const int voff = i * 64 + 32 * (hf ^ ((i >> 1) & 1));  // V rows swizzled (vrow_off)
                     const uint8_t* kc = kpool + row * 64 + 32 * hf;
                     const uint8_t* vc = vpool + row * 64 + 32 * hf;
                     cp_async16(st + off, kc, pol);
                     cp_async16(st + off + 16, kc + 16, pol);
-                    cp_async16(st + kOffV + off, vc, pol);
-                    cp_async16(st + kOffV + off + 16, vc + 16, pol);
+                    cp_async16(st + kOffV + voff, vc, pol);
+                    cp_async16(st + kOffV + voff + 16, vc + 16, pol);
                     cp_async4(st + (hf ? kOffVs : kOffKs) + 4 * i, (hf ? p.g.v_sz : p.g.k_sz) + row);
                 } else if (hf == 0) {
                     flag_error(p.err, kErrOOB);
@@ -273,11 +281,10 @@ __device__ __forceinline__ void stage_szf(CtaRing& R, const uint8_t* st, int war
 template <bool kLow>
 __device__ __forceinline__ void pv_chunk(float (&O)[8][4], const uint8_t* st, int gq, int tokA, int tokB, uint32_t b0,
                                          uint32_t b1, uint32_t b0l, uint32_t b1l) {
-    const uint8_t* vc = st + kOffV + 8 * gq;
-    const uint2 v00 = *reinterpret_cast<const uint2*>(vc + tokA * 64);
-    const uint2 v01 = *reinterpret_cast<const uint2*>(vc + tokB * 64);
-    const uint2 v10 = *reinterpret_cast<const uint2*>(vc + (8 + tokA) * 64);
-    const uint2 v11 = *reinterpret_cast<const uint2*>(vc + (8 + tokB) * 64);
+    const uint2 v00 = *reinterpret_cast<const uint2*>(st + vrow_off(tokA, 8 * gq));
+    const uint2 v01 = *reinterpret_cast<const uint2*>(st + vrow_off(tokB, 8 * gq));
+    const uint2 v10 = *reinterpret_cast<const uint2*>(st + vrow_off(8 + tokA, 8 * gq));
+    const uint2 v11 = *reinterpret_cast<const uint2*>(st + vrow_off(8 + tokB, 8 * gq));
 #pragma unroll
     for (int wq = 0; wq < 2; ++wq) {
         const uint32_t x00 = wq ? v00.y : v00.x, x01 = wq ? v01.y : v01.x;
