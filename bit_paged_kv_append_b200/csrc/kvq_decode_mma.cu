@@ -37,8 +37,8 @@
 //   G <= 4, tokens on M (decode_tok_kernel): q.K is D[16 tokens x 8 cols] =
 //     A[16 tokens x 32 dims] B[32 dims x 8 cols] on the int8 tensor path: A =
 //     codes as bytes (AND / shift-AND, 8 codes for 3 instructions), B = q' as
-//     16-bit fixed point per head, split into a signed high and low byte (the
-//     8 columns are 4 heads x {high, low}); the int32 accumulation is exact.
+//     23-bit fixed point per head in three signed bytes (n-tile 0: 4 heads x
+//     {high, middle}; n-tile 1: the low bytes); the int32 accumulation is exact.
 //     Every lane holds two real scores (no idle rows at G = 4), and the P.V B
 //     operand takes its 8 columns as 4 heads x {high, low part of p scale}, so
 //     the low part costs no extra mma; two shuffles move each score from the
@@ -63,7 +63,7 @@ constexpr int kOffVs = 2 * kCodeBytes + kChunk * 4;
 constexpr int kStageBytes = 2 * kCodeBytes + 2 * kChunk * 4;  // 2176
 constexpr float kTwo24 = 16777216.0f;  // a masked nibble c in an fp16 lane is the subnormal c * 2^-24
 constexpr float kTwo20 = 1048576.0f;   // ... and a masked high nibble is 16 c * 2^-24 = c * 2^-20
-constexpr int kQFix = 32639;           // |q| fixed point of the int8 tile: 256 hi + lo, hi, lo in [-128, 127]
+constexpr int kQFix = 8355711;  // |q_int| bound: 65536 hi + 256 mid + lo with hi, mid, lo in [-128, 127]
 constexpr uint32_t kFull = 0xffffffffu;
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -140,6 +140,22 @@ __device__ __forceinline__ int sigma(int n) { return n ^ ((n >> 2) & 1); }
 // set) that one 8-byte P.V load reads in each half-warp hit four distinct 32-byte
 // bank groups.
 __device__ __forceinline__ int vrow_off(int r, int b) { return kOffV + 64 * r + (b ^ ((r & 2) << 4)); }
+
+// q' in fixed point (23 bits: q_int = rint(q' kQFix / max|q'|)) as three balanced signed
+// bytes, q_int = 65536 hi + 256 mid + lo.  Fewer bits (16: two bytes) cost up to ~2e-3
+// of the output on keys with outlier channels; 23 bits cost ~5e-6.
+__device__ __forceinline__ void q_digits(int q, int& hi, int& mid, int& lo) {
+    q = min(max(q, -kQFix), kQFix);
+    lo = ((q + 128) & 255) - 128;
+    const int q1 = (q - lo) >> 8;  // exact
+    mid = ((q1 + 128) & 255) - 128;
+    hi = (q1 - mid) >> 8;          // exact, in [-127, 127]
+}
+
+// Score sum from the three digit partial sums (|each| < 2^18): 65536 hi + 256 mid + lo.
+__device__ __forceinline__ float q_dot(int dhi, int dmid, int dlo) {
+    return fmaf(float(dhi), 65536.0f, float(dmid * 256 + dlo));
+}
 
 // What a CTA keeps in shared memory for its warps' chunk streams.
 struct CtaRing {
@@ -364,9 +380,11 @@ __device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, C
 // G = 8: heads on M, fp16 q.K
 // =====================================================================================
 template <int G>
-__global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p) {
     __shared__ __align__(128) CtaRing R;
-    __shared__ uint32_t As[4 * 4 * 32];  // q.K A operand (4 x s8 per word) in fragment order: [k-step][reg][lane]
+    // q.K A operands (4 x s8 per word) in fragment order: m-tile 0 (rows hi | mid), [k-step][reg][lane];
+    // m-tile 1 (rows lo | zero), [k-step][even / odd dims][lane]
+    __shared__ uint32_t As[4 * 4 * 32 + 4 * 2 * 32];
     __shared__ float qsc_s[kMaxGroup], qsn_s[kMaxGroup];  // per head: fixed-point step, sum of q_int
 
     const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
@@ -374,13 +392,14 @@ __global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p)
     const int gq = lane >> 2, pq = lane & 3;  // mma group id / thread in group
     ChunkStream cs;
     if (!begin_split(p, R, cs, warp, lane, tid)) return;
-    for (int w = tid; w < 4 * 4 * 32; w += kThreads) As[w] = 0u;
+    for (int w = tid; w < 4 * 4 * 32 + 4 * 2 * 32; w += kThreads) As[w] = 0u;
     __syncthreads();
     const int nw = cs.nw, t1 = cs.t1;
 
-    // ---------------- q' as 16-bit fixed point per head, A fragment order ----------------
+    // ---------------- q' as 23-bit fixed point per head, A fragment order ----------------
     // k-step j, k-slot 4 pq + i (registers 0, 1) / 16 + 4 pq + i (registers 2, 3) stand for
-    // dim 32 pq + 8 j + 2 i (+ 1); rows 0..7 hold hi, rows 8..15 lo of q_int = 256 hi + lo.
+    // dim 32 pq + 8 j + 2 i (+ 1); m-tile 0: rows 0..7 hi, rows 8..15 mid; m-tile 1: rows
+    // 0..7 lo, rows 8..15 zero.
     for (int row = warp; row < G; row += kWarps) {
         float x[4];
         load_q_rotated(p, int64_t(s) * p.g.Hq + h * G + row, lane, x);
@@ -391,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p)
         int qi[4], isum = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            qi[c] = __float2int_rn(x[c] * inv);  // |qi| <= kQFix
+            qi[c] = min(max(__float2int_rn(x[c] * inv), -kQFix), kQFix);
             isum += qi[c];
         }
 #pragma unroll
@@ -401,14 +420,17 @@ __global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p)
             qsn_s[row] = float(isum);
         }
         uint8_t* A8 = reinterpret_cast<uint8_t*>(As);
+        uint8_t* A8lo = reinterpret_cast<uint8_t*>(As + 4 * 4 * 32);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int d = 4 * lane + c;
             const int dp = d >> 5, j = (d >> 3) & 3, i = (d >> 1) & 3, odd = d & 1;
-            const int hi = (qi[c] + 128) >> 8, lo = qi[c] - 256 * hi;  // both in [-128, 127]
-            const int lw = 4 * row + dp;                                // lane of row gq = row
+            int hi, mid, lo;
+            q_digits(qi[c], hi, mid, lo);
+            const int lw = 4 * row + dp;  // lane of row gq = row
             A8[((j * 4 + 2 * odd) * 32 + lw) * 4 + i] = uint8_t(hi);
-            A8[((j * 4 + 2 * odd + 1) * 32 + lw) * 4 + i] = uint8_t(lo);
+            A8[((j * 4 + 2 * odd + 1) * 32 + lw) * 4 + i] = uint8_t(mid);
+            A8lo[((j * 2 + odd) * 32 + lw) * 4 + i] = uint8_t(lo);
         }
     }
     // q only (never written by an append) so far; the cache after the previous grid
@@ -419,11 +441,14 @@ __global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p)
         cp_async_commit();
     }
     __syncthreads();
-    uint32_t A[4][4];
+    uint32_t A[4][4], Alo[4][2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < 4; ++j) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) A[j][r] = As[(j * 4 + r) * 32 + lane];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) Alo[j][r] = As[4 * 4 * 32 + (j * 2 + r) * 32 + lane];
+    }
     const float qsc = gq < G ? qsc_s[gq] : 0.0f, qsn = gq < G ? qsn_s[gq] : 0.0f;
 
     // ---------------- main loop over this warp's chunks ----------------
@@ -451,11 +476,16 @@ __global__ void __launch_bounds__(kThreads, 5) decode_mma_kernel(DecodeParams p)
         for (int tau = 0; tau < 2; ++tau) {
             const uint4 kw = *reinterpret_cast<const uint4*>(st + (8 * tau + tokK) * 64 + 16 * pq);
             const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
-            int D[4] = {0, 0, 0, 0};
+            int D[4] = {0, 0, 0, 0}, E[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) mma16832_s8u8(D, A[j], w[j] & 0x0F0F0F0Fu, (w[j] >> 4) & 0x0F0F0F0Fu);
-            C[tau][0] = float(D[0] * 256 + D[2]);  // head gq, column 2 pq; |S| < 2^26
-            C[tau][1] = float(D[1] * 256 + D[3]);  // head gq, column 2 pq + 1
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t b0 = w[j] & 0x0F0F0F0Fu, b1 = (w[j] >> 4) & 0x0F0F0F0Fu;
+                const uint32_t alo[4] = {Alo[j][0], 0u, Alo[j][1], 0u};
+                mma16832_s8u8(D, A[j], b0, b1);
+                mma16832_s8u8(E, alo, b0, b1);
+            }
+            C[tau][0] = q_dot(D[0], D[2], E[0]);  // head gq, column 2 pq
+            C[tau][1] = q_dot(D[1], D[3], E[1]);  // head gq, column 2 pq + 1
         }
         // A chunk whose 16 tokens all lie before the end and on valid pages needs no
         // per-token masks (the common case).
@@ -562,7 +592,9 @@ template <int G>
 __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p) {
     static_assert(G >= 1 && G <= 4, "tokens-on-M tile serves up to 4 query heads per KV head");
     __shared__ __align__(128) CtaRing R;
-    __shared__ uint32_t Bs[4 * 2 * 32];  // q.K B operand (4 x s8 per word) in fragment order: [k-step][reg][lane]
+    // q.K B operands (4 x s8 per word) in fragment order, [k-step][reg][lane]: n-tile 0
+    // (columns 2 head: hi, 2 head + 1: mid), n-tile 1 (columns 2 head: lo, odd columns zero)
+    __shared__ uint32_t Bs[2 * 4 * 2 * 32];
     __shared__ float qsc_s[4], qsn_s[4];  // per head: fixed-point step of q', sum of the fixed-point q'
 
     const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
@@ -570,14 +602,15 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
     const int gq = lane >> 2, pq = lane & 3;
     ChunkStream cs;
     if (!begin_split(p, R, cs, warp, lane, tid)) return;
-    for (int w = tid; w < 4 * 2 * 32; w += kThreads) Bs[w] = 0u;
+    for (int w = tid; w < 2 * 4 * 2 * 32; w += kThreads) Bs[w] = 0u;
     __syncthreads();
     const int nw = cs.nw, t1 = cs.t1;
 
-    // ---------------- q' as 16-bit fixed point per head, B fragment order ----------------
+    // ---------------- q' as 23-bit fixed point per head, B fragment order ----------------
     // k-step j, k-slot 4 pq + i (register 0) / 16 + 4 pq + i (register 1) stand for dim
     // 32 pq + 8 j + 2 i (+ 1): the low / high nibbles of bytes 16 pq + 4 j + i.
-    // Column n = 2 head + part: part 0 holds hi, part 1 lo of q_int = 256 hi + lo.
+    // n-tile 0, column 2 head + part: part 0 holds hi, part 1 mid; n-tile 1, column
+    // 2 head: lo.
     for (int row = warp; row < G; row += kWarps) {
         float x[4];
         load_q_rotated(p, int64_t(s) * p.g.Hq + h * G + row, lane, x);
@@ -588,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         int qi[4], isum = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            qi[c] = __float2int_rn(x[c] * inv);  // |qi| <= kQFix
+            qi[c] = min(max(__float2int_rn(x[c] * inv), -kQFix), kQFix);
             isum += qi[c];
         }
 #pragma unroll
@@ -598,13 +631,16 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
             qsn_s[row] = float(isum);
         }
         uint8_t* B8 = reinterpret_cast<uint8_t*>(Bs);
+        uint8_t* B8lo = reinterpret_cast<uint8_t*>(Bs + 4 * 2 * 32);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int d = 4 * lane + c;
             const int dp = d >> 5, j = (d >> 3) & 3, i = (d >> 1) & 3, r = d & 1;
-            const int hi = (qi[c] + 128) >> 8, lo = qi[c] - 256 * hi;  // both in [-128, 127]
+            int hi, mid, lo;
+            q_digits(qi[c], hi, mid, lo);
             B8[((j * 2 + r) * 32 + 4 * (2 * row) + dp) * 4 + i] = uint8_t(hi);
-            B8[((j * 2 + r) * 32 + 4 * (2 * row + 1) + dp) * 4 + i] = uint8_t(lo);
+            B8[((j * 2 + r) * 32 + 4 * (2 * row + 1) + dp) * 4 + i] = uint8_t(mid);
+            B8lo[((j * 2 + r) * 32 + 4 * (2 * row) + dp) * 4 + i] = uint8_t(lo);
         }
     }
     // q only (never written by an append) so far; the cache after the previous grid
@@ -615,11 +651,14 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         cp_async_commit();
     }
     __syncthreads();
-    uint32_t Bq[4][2];
+    uint32_t Bq[4][2], Blo[4][2];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) Bq[j][r] = Bs[(j * 2 + r) * 32 + lane];
+        for (int r = 0; r < 2; ++r) {
+            Bq[j][r] = Bs[(j * 2 + r) * 32 + lane];
+            Blo[j][r] = Bs[4 * 2 * 32 + (j * 2 + r) * 32 + lane];
+        }
 
     // ---------------- main loop over this warp's chunks ----------------
     // Thread (gq, pq) scores tokens tk, tk + 8 against head pq; heads >= G hold m = 0 and
@@ -653,14 +692,15 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         const uint4 k0 = *reinterpret_cast<const uint4*>(st + tk * 64 + 16 * pq);
         const uint4 k1 = *reinterpret_cast<const uint4*>(st + (tk + 8) * 64 + 16 * pq);
         const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-        int D[4] = {0, 0, 0, 0};
+        int D[4] = {0, 0, 0, 0}, E[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint32_t a[4] = {w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
                                    (w1[j] >> 4) & 0x0F0F0F0Fu};
             mma16832_u8s8(D, a, Bq[j][0], Bq[j][1]);
+            mma16832_u8s8(E, a, Blo[j][0], Blo[j][1]);
         }
-        const float S0 = float(D[0] * 256 + D[1]), S1 = float(D[2] * 256 + D[3]);  // |S| < 2^26
+        const float S0 = q_dot(D[0], D[1], E[0]), S1 = q_dot(D[2], D[3], E[2]);
         const float2 kz0 = R.szf[warp][0][tk], kz1 = R.szf[warp][0][tk + 8];
         const float v0 = qsc * fmaf(kz0.x, S0, kz0.y * qsn), v1 = qsc * fmaf(kz1.x, S1, kz1.y * qsn);
         const bool full = (tb + kChunk <= t1) && (vmask == 0xFFFFu);
