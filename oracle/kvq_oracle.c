@@ -44,8 +44,9 @@
  *     and max canonicalised to +0 first; inv = fl(1 / float(scale)) or 0 when
  *     scale is not positive; code = clamp(rint_even(fl(y - zero) * inv), 0, 15)
  *     where the product fl(y - zero) * inv is taken exactly (not rounded to
- *     fp32 before the rounding to an integer) and NaN goes to 0.  Dequantised
- *     value = code * scale + zero.
+ *     fp32 before the rounding to an integer).  A row holding a NaN has NaN
+ *     min and max: scale = zero = fp16 quiet NaN 0x7E00 and every code 0.
+ *     Dequantised value = code * scale + zero.
  *  R5 Packing: byte j holds code 2j in its low nibble and code 2j+1 in its
  *     high nibble.
  *  R6 Page layout: codes uint8 [pages, H_kv, page_size, D/2]; scale/zero as
@@ -150,6 +151,15 @@ void oracle_rotate_f64(double* x, int D, int b) {
 /* Quantise one (already rotated) row y[0..D) into D/2 packed bytes and an
  * (scale, zero) fp16 pair. */
 void oracle_quant_row(const float* y, int D, uint8_t* codes, uint16_t* scale_zero) {
+    /* a NaN anywhere makes the row's min and max NaN (reading): scale and zero are the
+     * fp16 quiet NaN 0x7E00 and every code is 0 */
+    for (int i = 0; i < D; i++) {
+        if (y[i] != y[i]) {
+            for (int j = 0; j < D / 2; j++) codes[j] = 0;
+            scale_zero[0] = scale_zero[1] = 0x7E00;
+            return;
+        }
+    }
     float mn = y[0], mx = y[0];
     for (int i = 1; i < D; i++) {
         if (y[i] < mn) mn = y[i];

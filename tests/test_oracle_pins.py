@@ -234,6 +234,16 @@ def test_quant_signed_zero_row_is_canonical():
     assert sz[0] == 0 and sz[1] == 0 and not codes.any()
 
 
+@pytest.mark.parametrize("where", [0, 77, 127])
+def test_quant_nan_row_is_all_zero_codes_with_nan_scale(where):
+    """A NaN anywhere in the row (reading: min and max are then NaN): every code 0, scale
+    and zero the fp16 quiet NaN 0x7E00; the position of the NaN does not matter."""
+    y = np.linspace(-2, 3, 128).astype(np.float32)
+    y[where] = np.nan
+    codes, sz = oracle.quant_row(y)
+    assert not codes.any() and sz[0] == 0x7E00 and sz[1] == 0x7E00
+
+
 def test_quant_rows_matches_rotate_then_quant():
     """quant_rows(x, b) == quant_row(rotate_f32(x)) row by row; b = 0 means no rotation."""
     rng = np.random.default_rng(5)
