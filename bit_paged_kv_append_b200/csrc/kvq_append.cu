@@ -151,22 +151,52 @@ __device__ __forceinline__ void quantise_pack(const float2 (&R)[64], float zf, f
     }
 }
 
+// min / max that return NaN when any input is NaN
+__device__ __forceinline__ float min_nan(float a, float b) {
+    float d;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+__device__ __forceinline__ float min3_nan(float a, float b, float c) {
+    float d;
+    asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Token-wise asymmetric INT4 of one row: writes 64 bytes of codes and the
-// (scale, zero) word.
+// (scale, zero) word.  A NaN anywhere in the row makes its min and max NaN:
+// every code 0, scale = zero = fp16 quiet NaN.
 __device__ __forceinline__ void quantise_store(const float2 (&R)[64], uint8_t* codes_dst, uint32_t* sz_dst) {
     float mn4[4], mx4[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        mn4[k] = fminf(R[k].x, R[k].y);
-        mx4[k] = fmaxf(R[k].x, R[k].y);
+        mn4[k] = min_nan(R[k].x, R[k].y);
+        mx4[k] = max_nan(R[k].x, R[k].y);
     }
 #pragma unroll
     for (int i = 4; i < 64; ++i) {
-        mn4[i & 3] = min3(mn4[i & 3], R[i].x, R[i].y);
-        mx4[i & 3] = max3(mx4[i & 3], R[i].x, R[i].y);
+        mn4[i & 3] = min3_nan(mn4[i & 3], R[i].x, R[i].y);
+        mx4[i & 3] = max3_nan(mx4[i & 3], R[i].x, R[i].y);
     }
-    float mn = min3(mn4[0], mn4[1], fminf(mn4[2], mn4[3]));
-    float mx = max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+    float mn = min3_nan(mn4[0], mn4[1], min_nan(mn4[2], mn4[3]));
+    float mx = max3_nan(mx4[0], mx4[1], max_nan(mx4[2], mx4[3]));
+    if (mn != mn) {
+        const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        st_global_v8(codes_dst, z);
+        st_global_v8(codes_dst + 32, z);
+        *sz_dst = 0x7E007E00u;
+        return;
+    }
     mn = __fadd_rn(mn, 0.0f);  // -0 + +0 = +0: canonical signed zero
     mx = __fadd_rn(mx, 0.0f);
     const float range = __fsub_rn(mx, mn);
@@ -177,7 +207,7 @@ __device__ __forceinline__ void quantise_store(const float2 (&R)[64], uint8_t* c
     const float zf = __half2float(zh);
     const float inv = sf > 0.0f ? __frcp_rn(sf) : 0.0f;
     // The quantiser is monotone in y, so the row's extreme codes decide whether any
-    // element needs clamping; NaN fails both tests and takes the clamped path.
+    // element needs clamping (an infinite scale or zero fails the test).
     const float umin = __fmaf_rn(__fsub_rn(mn, zf), inv, kMagic);
     const float umax = __fmaf_rn(__fsub_rn(mx, zf), inv, kMagic);
     const bool in_range = (umin >= kMagic) && (umax <= kMagic + 15.0f);

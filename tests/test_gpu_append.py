@@ -97,6 +97,10 @@ def _special_rows(H):
     rows.append(off)
     levels = (torch.arange(128) % 16).float() * 0.5
     rows.append(levels)
+    for where in (0, 77):  # a NaN anywhere: every code 0, scale = zero = fp16 NaN
+        nan_row = torch.linspace(-2, 3, 128)
+        nan_row[where] = float("nan")
+        rows.append(nan_row)
     x = torch.stack(rows)  # [R, 128]
     reps = -(-(H * 40) // x.shape[0])
     return x.repeat(reps, 1)[: H * 40].reshape(40, H, 128).to(torch.bfloat16)
@@ -105,7 +109,8 @@ def _special_rows(H):
 @pytest.mark.parametrize("b,rv", [(0, False), (16, True), (128, True)])
 def test_append_special_values(b, rv):
     """Constant rows, signed zeros, fp16 overflow of scale or zero, subnormal fp16 scales,
-    rows far from zero and exact 16-level rows take the same decisions as the oracle."""
+    rows far from zero, exact 16-level rows and rows holding a NaN take the same decisions
+    as the oracle."""
     mode = kvq.KV_INT4 if b == 0 else kvq.KV_INT4_BDR
     c = make_case(mode, b, rv, [40], WL0, seed=5)
     k = _special_rows(8)
