@@ -55,7 +55,7 @@ kv_status kv_create_paged(const kv_desc* d, kv_cache** out) {
     if (d->mode != KV_BF16 && (!d->k_sz || !d->v_sz || !aligned(d->k_sz, 16) || !aligned(d->v_sz, 16)))
         return KV_ERR_INVALID;
     const int64_t rows = int64_t(d->num_pages) * d->num_kv_heads * d->page_size;
-    if (rows > (int64_t(1) << 40)) return KV_ERR_INVALID;
+    if (rows >= (int64_t(1) << 32)) return KV_ERR_INVALID;  // slot indices are 32-bit in the kernels
 
     kv_cache* c = new (std::nothrow) kv_cache();
     if (!c) return KV_ERR_INVALID;

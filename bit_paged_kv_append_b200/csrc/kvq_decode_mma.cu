@@ -104,6 +104,10 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint64_t 
                  "l"(pol)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async16_s(uint32_t dst, const void* src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
@@ -164,59 +168,82 @@ struct CtaRing {
     float2 szf[kWarps][2][kChunk];      // (scale, offset) of the current chunk: [warp][K / V][token]
 };
 
-// One warp's 16-token chunks of its split: page lookups (one page-table entry per
-// lane, 32 chunks a window) and the copies of chunk iw into a ring stage.
+// One warp's 16-token chunks of its split: pool rows (one page-table lookup per lane,
+// 32 chunks a window) and the copies of chunk iw into a ring stage.
 struct ChunkStream {
     CtaRing* r;
     const int32_t* pt;  // this sequence's page-table row
     int t0, t1, nw, warp, lane, h;
     bool fast;          // page size a multiple of 16: a chunk is 16 consecutive slots of one page
     uint64_t pol;
-    int win, mypage;
+    int win;
+    uint32_t myrow;     // pool row of this lane's chunk of the window, or kNoRow
+    // per-lane sources (fast path): byte 16 lane of the K / V code blocks, and the
+    // scale/zero words lanes 0..7 copy (4 K words per lane for lanes 0..3, V for 4..7)
+    const uint8_t* kc;
+    const uint8_t* vc;
+    const uint32_t* sz;
+    uint32_t dst0;      // shared address of this lane's K destination in slot 0
 
-    __device__ __forceinline__ int page_of(const DecodeParams& p, int iw) {
+    static constexpr uint32_t kNoRow = 0xFFFFFFFFu;
+
+    __device__ __forceinline__ void init(const DecodeParams& p) {
+        win = -1;
+        myrow = kNoRow;
+        kc = static_cast<const uint8_t*>(p.g.k_pool) + 16 * lane;
+        vc = static_cast<const uint8_t*>(p.g.v_pool) + 16 * lane;
+        sz = (lane < 4 ? p.g.k_sz : p.g.v_sz) + 4 * (lane & 3);
+        dst0 = smem_u32(r->stage[warp][0]) + 16 * lane;
+    }
+
+    // Pool row (page H + h) ps + slot of chunk iw's first token (all lanes; kNoRow for a
+    // bad page, flagged once when its window is loaded).
+    __device__ __forceinline__ uint32_t row_of(const DecodeParams& p, int iw) {
         if ((iw >> 5) != win) {
             win = iw >> 5;
             const int ci = 32 * win + lane;
-            mypage = ci < nw ? __ldg(pt + page_of_pos(p, t0 + (warp + kWarps * ci) * kChunk)) : -1;
+            myrow = kNoRow;
+            if (ci < nw) {
+                const int tb = t0 + (warp + kWarps * ci) * kChunk;
+                const int page = __ldg(pt + page_of_pos(p, tb));
+                if (page >= 0 && page < p.g.num_pages)
+                    myrow = (uint32_t(page) * uint32_t(p.g.H) + uint32_t(h)) * uint32_t(p.g.page_size) +
+                            uint32_t(slot_of_pos(p, tb));
+                else
+                    flag_error(p.err, kErrOOB);
+            }
         }
-        return __shfl_sync(kFull, mypage, iw & 31);
+        return __shfl_sync(kFull, myrow, iw & 31);
     }
 
     // Copies of chunk iw into ring slot by all 32 lanes (16-byte cp.async, no divergent
-    // issuer), then one commit: the stream always holds one copy group per chunk slot.
+    // issuer); the caller commits one copy group per chunk slot.
     __device__ __forceinline__ void issue(const DecodeParams& p, int iw, int slot) {
-        uint8_t* st = r->stage[warp][slot];
-        const int tb = t0 + (warp + kWarps * iw) * kChunk;
-        const uint8_t* kpool = static_cast<const uint8_t*>(p.g.k_pool);
-        const uint8_t* vpool = static_cast<const uint8_t*>(p.g.v_pool);
-        const int H = p.g.H, ps = p.g.page_size;
         if (fast) {
             // 16 consecutive slots of one page: 1 KiB of K codes, 1 KiB of V codes, 64 B of
             // scale/zero words each; lane L copies bytes 16 L and 512 + 16 L of both code
-            // blocks, lanes 0..3 / 4..7 the K / V scale/zero words
-            const int page = page_of(p, iw);
-            const bool ok = page >= 0 && page < p.g.num_pages;
+            // blocks (V rows swizzled, vrow_off), lanes 0..3 / 4..7 the K / V words
+            const uint32_t row = row_of(p, iw);
+            const bool ok = row != kNoRow;
             if (ok) {
-                const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, tb);
-                const uint8_t* kc = kpool + row * 64 + 16 * lane;
-                const uint8_t* vc = vpool + row * 64 + 16 * lane;
-                const int vu = 16 * (lane ^ ((lane >> 2) & 2));  // V rows swizzled (vrow_off)
-                cp_async16(st + 16 * lane, kc, pol);
-                cp_async16(st + 512 + 16 * lane, kc + 512, pol);
-                cp_async16(st + kOffV + vu, vc, pol);
-                cp_async16(st + kOffV + 512 + vu, vc + 512, pol);
-                if (lane < 8) {
-                    const uint32_t* sz = (lane < 4 ? p.g.k_sz : p.g.v_sz) + row + 4 * (lane & 3);
-                    cp_async16(st + kOffKs + 16 * lane, sz, pol);  // V words follow the K words
-                }
-            } else if (lane == 0) {
-                flag_error(p.err, kErrOOB);
+                const uint32_t d = dst0 + uint32_t(slot) * kStageBytes;
+                const int vsw = 16 * ((lane >> 2) & 2);  // this lane's V unit moves by 32 bytes
+                const uint8_t* ks = kc + size_t(row) * 64;
+                const uint8_t* vs = vc + size_t(row) * 64;
+                cp_async16_s(d, ks, pol);
+                cp_async16_s(d + 512, ks + 512, pol);
+                cp_async16_s((d + kOffV) ^ vsw, vs, pol);
+                cp_async16_s(((d + kOffV) ^ vsw) + 512, vs + 512, pol);
+                if (lane < 8) cp_async16_s(d + kOffKs, sz + row, pol);  // V words follow the K words
             }
-            if (lane == 0) r->mask[warp][slot] = ok ? 0xFFFFu : 0u;
+            r->mask[warp][slot] = ok ? 0xFFFFu : 0u;  // the same value from every lane
         } else {
             // gather: lane L copies half L & 1 of token tb + (L >> 1)'s K and V code rows and
             // its K (even L) or V (odd L) scale/zero word
+            uint8_t* st = r->stage[warp][slot];
+            const int tb = t0 + (warp + kWarps * iw) * kChunk;
+            const uint8_t* kpool = static_cast<const uint8_t*>(p.g.k_pool);
+            const uint8_t* vpool = static_cast<const uint8_t*>(p.g.v_pool);
             const int i = lane >> 1, hf = lane & 1;
             const int t = tb + i;
             bool ok = false;
@@ -224,15 +251,15 @@ struct ChunkStream {
                 const int page = __ldg(pt + page_of_pos(p, t));
                 ok = page >= 0 && page < p.g.num_pages;
                 if (ok) {
-                    const int64_t row = (int64_t(page) * H + h) * ps + slot_of_pos(p, t);
+                    const int64_t row = (int64_t(page) * p.g.H + h) * p.g.page_size + slot_of_pos(p, t);
                     const int off = i * 64 + 32 * hf;
                     const int voff = i * 64 + 32 * (hf ^ ((i >> 1) & 1));  // V rows swizzled (vrow_off)
-                    const uint8_t* kc = kpool + row * 64 + 32 * hf;
-                    const uint8_t* vc = vpool + row * 64 + 32 * hf;
-                    cp_async16(st + off, kc, pol);
-                    cp_async16(st + off + 16, kc + 16, pol);
-                    cp_async16(st + kOffV + voff, vc, pol);
-                    cp_async16(st + kOffV + voff + 16, vc + 16, pol);
+                    const uint8_t* kcp = kpool + row * 64 + 32 * hf;
+                    const uint8_t* vcp = vpool + row * 64 + 32 * hf;
+                    cp_async16(st + off, kcp, pol);
+                    cp_async16(st + off + 16, kcp + 16, pol);
+                    cp_async16(st + kOffV + voff, vcp, pol);
+                    cp_async16(st + kOffV + voff + 16, vcp + 16, pol);
                     cp_async4(st + (hf ? kOffVs : kOffKs) + 4 * i, (hf ? p.g.v_sz : p.g.k_sz) + row);
                 } else if (hf == 0) {
                     flag_error(p.err, kErrOOB);
@@ -371,8 +398,7 @@ __device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, C
     cs.h = h;
     cs.fast = (p.g.page_size % kChunk) == 0;
     cs.pol = policy_evict_first();
-    cs.win = -1;
-    cs.mypage = -1;
+    cs.init(p);
     return true;
 }
 

@@ -80,7 +80,7 @@ typedef enum {
 } kv_mode;
 
 typedef struct {
-    int num_pages;    /* pages in each pool */
+    int num_pages;    /* pages in each pool; num_pages * num_kv_heads * page_size < 2^32 */
     int page_size;    /* tokens per page, 1..1024 */
     int num_kv_heads; /* H_kv: 1, 2, 4, 8, 16 or 32 */
     int num_q_heads;  /* H_q = G * H_kv with G in {1, 2, 4, 8} */
