@@ -280,6 +280,46 @@ def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False):
             "launches_per_step": len(w.appends) + 2}
 
 
+def exact_attention(k, v, q, lengths, H, Hq):
+    """float64 attention of q over the unquantised bf16 K/V rows (sequence-major, positions 0..L-1):
+    the values the quantised caches approximate (no cache, no quantisation, no rotation)."""
+    kf = k.float().cpu().numpy().astype(np.float64)
+    vf = v.float().cpu().numpy().astype(np.float64)
+    qf = q.float().cpu().numpy().astype(np.float64)
+    G = Hq // H
+    out = np.zeros((len(lengths), Hq, 128))
+    off = 0
+    for s, L in enumerate(lengths):
+        Ks, Vs = kf[off:off + L], vf[off:off + L]
+        off += L
+        for j in range(Hq):
+            sc = Ks[:, j // G] @ qf[s, j] / np.sqrt(128.0)
+            p = np.exp(sc - sc.max())
+            out[s, j] = (p @ Vs[:, j // G]) / p.sum()
+    return out
+
+
+def accuracy_study(w: Workload, device):
+    """Attention-output error of every cache variant (append + decode through the library, fp32
+    output) against exact float64 attention on the unquantised rows, per (sequence, query head)
+    row: max |o - r| / max |r|.  Whole sequences appended from position 0 (batch16, single256)."""
+    k, v, ts, tp = w.appends[0]
+    ref = exact_attention(k, v, w.q, w.dec_lens, w.H, w.Hq)
+    den = np.maximum(np.abs(ref).max(axis=-1), 1e-30)
+    res = {}
+    for name, mode, b, rv in VARIANTS:
+        cache = kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0)
+        cache.append(k, v, ts, tp, w.page_table)
+        out = cache.decode(w.q, w.seq_lens, w.dec_pt, w.max_len, out_fp32=True)
+        status = cache.get_error()
+        cache.close()
+        if status != kvq.KV_OK:
+            raise RuntimeError(f"device error in the accuracy study: {kvq.status_string(status)}")
+        err = np.abs(out.cpu().numpy().astype(np.float64) - ref).max(axis=-1) / den
+        res[name] = {"max_rel": float(err.max()), "mean_rel": float(err.mean())}
+    return res
+
+
 def run_e2e(w: Workload, mode, b, rv, steps, warmup, device):
     """Same step through the C ABI with pinned HOST inputs: H2D copies of the step's inputs and a
     D2H read of the attention output are inside the timed region (CUDA events, launching stream)."""
@@ -410,6 +450,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-accuracy", action="store_true")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -442,6 +483,10 @@ def main():
                            "decode_gbs": w.decode_bytes(mode) / (r["decode_ms"] / 1e3) / 1e9,
                            "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3}
         sweep["bdr128_k_over_int4_append"] = sweep["bdr128_k"]["append_tok_per_s"] / sweep["int4"]["append_tok_per_s"]
+
+    accuracy = None
+    if not args.no_accuracy and args.workload in ("batch16", "single256"):
+        accuracy = accuracy_study(w, device)
 
     e2e_ms, h2d, d2h = run_e2e(w, hmode, hb, hrv, max(20, min(200, args.steps // 20)), args.warmup, device)
     e2e_ms = reduce_over_ranks(e2e_ms, "max", device)
@@ -486,6 +531,9 @@ def main():
     }
     if sweep:
         line["sweep"] = sweep
+    if accuracy:
+        line["accuracy"] = {"vs": "exact float64 attention on the unquantised bf16 K/V",
+                            "metric": "per (sequence, query head) row max|o-r|/max|r|", **accuracy}
     if rank == 0 and world == 1 and not args.no_cpu:
         c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=min(w.tokens_per_step, 20000),
                                                  row_budget=8)
