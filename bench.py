@@ -365,39 +365,46 @@ def run_e2e(w: Workload, mode, b, rv, steps, warmup, device):
 
 # --------------------------------------------------------------------------- oracle (CPU)
 
-def oracle_unit_costs(w: Workload, mode, b, rv, tok_budget: int, row_budget: int, seed=0):
+def oracle_unit_costs(w: Workload, mode, b, rv, tok_budget: int, row_budget: int, seed=0, dec_seqs: int = 1,
+                      reps: int = 1):
     """Seconds per appended token and per (cached token x query head) of the CPU oracle, measured
-    on a bounded sample shaped like the workload (tok_budget appended tokens; row_budget decode
-    rows over a sequence of the workload's mean decoded length)."""
+    on a bounded sample shaped like the workload: tok_budget appended tokens, and row_budget
+    query-head rows of each of dec_seqs sequences of the workload's mean decoded length; the
+    whole sample is run reps times (seeds seed .. seed + reps - 1) and the times summed."""
     import oracle
 
     H, ps = w.H, w.ps
     bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
     n = max(1, tok_budget)
-    k, v = synth.make_kv(n, w.wl, seed)
     Ls = int(min(max(np.mean(w.dec_lens), 16), 32768))
-    cap = max(n, Ls)
-    pt, P = synth.make_page_table([cap], ps, seed)
-    if mode == kvq.KV_BF16:
-        kp = np.zeros((P, H, ps, 128), np.uint16)
-        ks = np.zeros(1, np.uint16)
-    else:
-        kp = np.zeros((P, H, ps, 64), np.uint8)
-        ks = np.zeros((P, H, ps, 2), np.uint16)
-    vp, vs = kp.copy(), ks.copy()
-    ts, tp = synth.append_positions([n])
-    t0 = time.perf_counter()
-    oracle.append(mode, b, rv, kp, vp, ks, vs, bits(k), bits(v), ts.numpy(), tp.numpy(), pt.numpy())
-    c_app = (time.perf_counter() - t0) / n
-    q = synth.make_q(1, w.Hq, 128, seed)
     r = max(1, min(row_budget, w.Hq))
-    rows = [(0, j) for j in range(r)]
-    t0 = time.perf_counter()
-    oracle.decode(mode, b, rv, kp, vp, ks, vs, bits(q), np.array([Ls]), pt.numpy(), H, rows=rows)
-    c_dec = (time.perf_counter() - t0) / (r * Ls)
-    sample = (f"oracle append of {n} tokens and decode of {r} query-head rows over {Ls} cached tokens, "
-              f"1 thread; per-unit costs scaled to one step ({w.tokens_per_step} tokens appended, "
-              f"{sum(w.dec_lens) * w.Hq} (token x query head) decoded)")
+    nd = max(1, dec_seqs)
+    t_app = t_dec = 0.0
+    for rep in range(reps):
+        sd = seed + rep
+        k, v = synth.make_kv(n, w.wl, sd)
+        pt, P = synth.make_page_table([max(n, Ls)] + [Ls] * (nd - 1), ps, sd)
+        if mode == kvq.KV_BF16:
+            kp = np.zeros((P, H, ps, 128), np.uint16)
+            ks = np.zeros(1, np.uint16)
+        else:
+            kp = np.zeros((P, H, ps, 64), np.uint8)
+            ks = np.zeros((P, H, ps, 2), np.uint16)
+        vp, vs = kp.copy(), ks.copy()
+        ts, tp = synth.append_positions([n])
+        t0 = time.perf_counter()
+        oracle.append(mode, b, rv, kp, vp, ks, vs, bits(k), bits(v), ts.numpy(), tp.numpy(), pt.numpy())
+        t_app += time.perf_counter() - t0
+        q = synth.make_q(nd, w.Hq, 128, sd)
+        rows = [(s, j) for s in range(nd) for j in range(r)]
+        t0 = time.perf_counter()
+        oracle.decode(mode, b, rv, kp, vp, ks, vs, bits(q), np.array([Ls] * nd), pt.numpy(), H, rows=rows)
+        t_dec += time.perf_counter() - t0
+    c_app = t_app / (n * reps)
+    c_dec = t_dec / (r * nd * Ls * reps)
+    sample = (f"{reps} x (oracle append of {n} tokens and decode of {r} query-head rows of {nd} sequence(s) "
+              f"over {Ls} cached tokens), 1 thread, {t_app + t_dec:.1f} s; per-unit costs scaled to one step "
+              f"({w.tokens_per_step} tokens appended, {sum(w.dec_lens) * w.Hq} (token x query head) decoded)")
     return c_app, c_dec, sample
 
 
@@ -535,8 +542,12 @@ def main():
         line["accuracy"] = {"vs": "exact float64 attention on the unquantised bf16 K/V",
                             "metric": "per (sequence, query head) row max|o-r|/max|r|", **accuracy}
     if rank == 0 and world == 1 and not args.no_cpu:
-        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=min(w.tokens_per_step, 20000),
-                                                 row_budget=8)
+        # about one step's worth of oracle work per repetition for batch16 (~4 s), bounded for the
+        # large workloads; 3 repetitions: ~10-15 s of host CPU
+        Ls = int(min(max(np.mean(w.dec_lens), 16), 32768))
+        nd = max(1, min(w.dec_B, 16, (1 << 20) // (w.Hq * Ls)))
+        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=min(w.tokens_per_step, 40960),
+                                                 row_budget=w.Hq, dec_seqs=nd, reps=3)
         line["cpu_baseline"] = {"value": w.tokens_per_step / oracle_step_seconds(w, c_app, c_dec),
                                 "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
     if rank == 0:
