@@ -351,6 +351,24 @@ __device__ __forceinline__ void pv_chunk(float (&O)[8][4], const uint8_t* st, in
     }
 }
 
+// Merge scratch mo [warp][G][128]: each 16-byte chunk of a head's row is stored at chunk
+// c ^ mo_swz(g), so the four 16-byte stores per lane of a 16-dim segment (the 8 lanes of
+// one store phase: two segments x four heads) hit distinct bank groups.
+template <int G>
+__device__ __forceinline__ int mo_swz(int g) { return G == 8 ? (g >> 1) & 3 : g & 3; }
+template <int G>
+__device__ __forceinline__ int mo_idx(int row, int g, int d) {
+    return row * kHeadDim + ((((d >> 2) ^ mo_swz<G>(g))) << 2) + (d & 3);
+}
+// dims 16 gq .. 16 gq + 15 of head g (v[i] = dim 16 gq + i) into the merge scratch row
+template <int G>
+__device__ __forceinline__ void mo_store16(float* mo, int row, int g, int gq, const float (&v)[16]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<float4*>(mo + mo_idx<G>(row, g, 16 * gq + 4 * c)) =
+            make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
 // Merge the 4 warps' partial states (mo [warp][G][128] outputs incl. the offset
 // term, mm / ml [warp][G] max and weight sum) and store the split's partial rows.
 template <int G>
@@ -366,7 +384,7 @@ __device__ __forceinline__ void store_partials(const DecodeParams& p, const floa
         for (int w = 0; w < kWarps; ++w) {
             const float mw = mm[w * G + g];
             const float f = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - M);
-            acc += f * mo[(w * G + g) * kHeadDim + tid];
+            acc += f * mo[mo_idx<G>(w * G + g, g, tid)];
             lt += f * ml[w * G + g];
         }
         const int64_t r = partial_row(p, s, k, h * G + g);
@@ -591,17 +609,23 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
     float* mm = mo + kWarps * G * kHeadDim;                   // [warp][G]
     float* ml = mm + kWarps * G;                              // [warp][G]
     const int h0 = 2 * pq, h1 = 2 * pq + 1;
+    if (h0 < G) {
+        float v[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int d = 16 * gq + 2 * j;
-        if (h0 < G) {
-            mo[(warp * G + h0) * kHeadDim + d] = O[j][0] * kTwo24 + Z0;
-            mo[(warp * G + h0) * kHeadDim + d + 1] = O[j][2] * kTwo20 + Z0;
+        for (int j = 0; j < 8; ++j) {
+            v[2 * j] = O[j][0] * kTwo24 + Z0;
+            v[2 * j + 1] = O[j][2] * kTwo20 + Z0;
         }
-        if (h1 < G) {
-            mo[(warp * G + h1) * kHeadDim + d] = O[j][1] * kTwo24 + Z1;
-            mo[(warp * G + h1) * kHeadDim + d + 1] = O[j][3] * kTwo20 + Z1;
+        mo_store16<G>(mo, warp * G + h0, h0, gq, v);
+    }
+    if (h1 < G) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            v[2 * j] = O[j][1] * kTwo24 + Z1;
+            v[2 * j + 1] = O[j][3] * kTwo20 + Z1;
         }
+        mo_store16<G>(mo, warp * G + h1, h1, gq, v);
     }
     if (pq == 0 && gq < G) {
         mm[warp * G + gq] = m;
@@ -794,12 +818,13 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
     float* mm = mo + kWarps * G * kHeadDim;                   // [warp][G]
     float* ml = mm + kWarps * G;                              // [warp][G]
     if (hv) {
+        float v[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const int d = 16 * gq + 2 * j;
-            mo[(warp * G + pq) * kHeadDim + d] = (O[j][0] + O[j][1]) * kTwo24 + Z;
-            mo[(warp * G + pq) * kHeadDim + d + 1] = (O[j][2] + O[j][3]) * kTwo20 + Z;
+            v[2 * j] = (O[j][0] + O[j][1]) * kTwo24 + Z;
+            v[2 * j + 1] = (O[j][2] + O[j][3]) * kTwo20 + Z;
         }
+        mo_store16<G>(mo, warp * G + pq, pq, gq, v);
         if (gq == 0) {
             mm[warp * G + pq] = m;
             ml[warp * G + pq] = l;
