@@ -148,6 +148,15 @@ def make_page_table(capacities: list[int], page_size: int, seed: int, spare_page
     return pt, num_pages
 
 
+def rope_table(positions: int, head_dim: int = 128, base: float = 1_000_000.0) -> torch.Tensor:
+    """A rotary-embedding input table, float32 [positions, head_dim/2, 2] = (cos, sin) of angle
+    pos * base^(-2i/head_dim) (the usual frequencies; computed in float64, rounded once)."""
+    i = torch.arange(head_dim // 2, dtype=torch.float64)
+    theta = base ** (-2.0 * i / head_dim)
+    ang = torch.arange(positions, dtype=torch.float64)[:, None] * theta[None, :]
+    return torch.stack([torch.cos(ang), torch.sin(ang)], dim=-1).to(torch.float32).contiguous()
+
+
 def append_positions(lengths: list[int], starts: list[int] | None = None):
     """Flattened (tok_seq, tok_pos) int32 for appending lengths[s] tokens to sequence s at starts[s]."""
     starts = starts or [0] * len(lengths)

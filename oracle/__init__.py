@@ -59,10 +59,11 @@ def _load():
         lib.oracle_quant_rows.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P]
         lib.oracle_append.restype = i64
         lib.oracle_append.argtypes = [ctypes.c_int] * 7 + [P] * 6 + [ctypes.c_int, P, P, P, ctypes.c_int,
-                                                                     ctypes.c_int]
+                                                                     ctypes.c_int, P, ctypes.c_int]
         lib.oracle_decode.restype = i64
         lib.oracle_decode.argtypes = [ctypes.c_int] * 8 + [P] * 7 + [ctypes.c_int, ctypes.c_int, P,
-                                                                     ctypes.c_int, P]
+                                                                     ctypes.c_int, P, P, ctypes.c_int]
+        lib.oracle_rope_f32.argtypes = [P, ctypes.c_int, P]
         _lib = lib
     return _lib
 
@@ -132,12 +133,29 @@ def unpack_codes(codes: np.ndarray) -> np.ndarray:
     return np.stack([lo, hi], axis=-1).reshape(codes.shape[:-1] + (codes.shape[-1] * 2,))
 
 
+def _rope_args(rope):
+    if rope is None:
+        return None, None, 0
+    r = np.ascontiguousarray(rope, dtype=np.float32)
+    return r, _ptr(r), r.shape[0]
+
+
+def rope_f32(x: np.ndarray, cs: np.ndarray) -> np.ndarray:
+    """Rotate-half RoPE of rows x (float32 [n, D]) with one table row cs (float32 [D/2, 2] = (cos, sin))."""
+    x = np.ascontiguousarray(x, dtype=np.float32).copy()
+    c = np.ascontiguousarray(cs, dtype=np.float32)
+    for r in range(x.shape[0]):
+        _load().oracle_rope_f32(_ptr(x[r]), x.shape[1], _ptr(c))
+    return x
+
+
 def append(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz, k_bits, v_bits,
-           tok_seq, tok_pos, page_table) -> int:
+           tok_seq, tok_pos, page_table, rope=None) -> int:
     """Append tokens into the pools in place (numpy arrays); returns the skipped-token count.
 
     Pools: INT4 uint8 [P, H, ps, D/2] (+ sz uint16 [P, H, ps, 2]); BF16 uint16 [P, H, ps, D].
     k_bits/v_bits: bf16 bits uint16 [T, H, D]; page_table int32 [num_seqs, pt_stride].
+    rope: optional float32 [positions, D/2, 2] (cos, sin) table that turns the keys first.
     """
     P, H, ps = k_pool.shape[:3]
     D = k_bits.shape[-1]
@@ -145,18 +163,20 @@ def append(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz
     pt = np.ascontiguousarray(page_table, dtype=np.int32)
     ts = np.ascontiguousarray(tok_seq, dtype=np.int32)
     tp = np.ascontiguousarray(tok_pos, dtype=np.int32)
+    keep, rp, rn = _rope_args(rope)
     return int(_load().oracle_append(mode, bdr_block, int(rotate_v), P, ps, H, D, _ptr(k_pool), _ptr(v_pool),
                                      _ptr(k_sz), _ptr(v_sz), _ptr(np.ascontiguousarray(k_bits)),
                                      _ptr(np.ascontiguousarray(v_bits)), T, _ptr(ts), _ptr(tp), _ptr(pt),
-                                     pt.shape[1], pt.shape[0]))
+                                     pt.shape[1], pt.shape[0], rp, rn))
 
 
 def decode(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz, q_bits, seq_lens,
-           page_table, num_kv_heads: int, rows=None):
+           page_table, num_kv_heads: int, rows=None, rope=None):
     """Paged GQA decode attention in float64.
 
     q_bits: bf16 bits uint16 [B, Hq, D].  rows: optional int array [(seq, qhead), ...]; when None all
-    B*Hq rows are computed.  Returns (out float64 [n, D] or [B, Hq, D], skipped-token count).
+    B*Hq rows are computed.  rope: optional float32 [positions, D/2, 2] table turning q at position
+    seq_len - 1.  Returns (out float64 [n, D] or [B, Hq, D], skipped-token count).
     """
     P = k_pool.shape[0]
     ps = k_pool.shape[2]
@@ -170,9 +190,10 @@ def decode(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz
         rws = None
         n = B * Hq
     out = np.empty((n, D), dtype=np.float64)
+    keep, rp, rn = _rope_args(rope)
     skipped = _load().oracle_decode(mode, bdr_block, int(rotate_v), P, ps, num_kv_heads, Hq, D, _ptr(k_pool),
                                     _ptr(v_pool), _ptr(k_sz), _ptr(v_sz), _ptr(np.ascontiguousarray(q_bits)),
-                                    _ptr(sl), _ptr(pt), pt.shape[1], B, _ptr(rws), n, _ptr(out))
+                                    _ptr(sl), _ptr(pt), pt.shape[1], B, _ptr(rws), n, _ptr(out), rp, rn)
     if rows is None:
         out = out.reshape(B, Hq, D)
     return out, int(skipped)

@@ -47,6 +47,10 @@
  *     fp32 before the rounding to an integer).  A row holding a NaN has NaN
  *     min and max: scale = zero = fp16 quiet NaN 0x7E00 and every code 0.
  *     Dequantised value = code * scale + zero.
+ *  Fused RoPE (optional): a caller-given table of (cos, sin) per position and
+ *     rotate-half pair turns the keys (fp32, before the block rotation; BF16
+ *     pages store the turned row rounded to bf16) and the query, at position
+ *     seq_len - 1, the newest token; positions outside the table are skipped.
  *  R5 Packing: byte j holds code 2j in its low nibble and code 2j+1 in its
  *     high nibble.
  *  R6 Page layout: codes uint8 [pages, H_kv, page_size, D/2]; scale/zero as
@@ -106,6 +110,31 @@ static float rb_f32(int b) { return (float)(1.0 / sqrt((double)b)); }
 
 /* In-place fp32 fast Walsh-Hadamard transform of each length-b block of x[0..D),
  * stages in increasing stride; normalised by r_b when normalise != 0. */
+/* fp32 -> bf16 bits, round to nearest even; NaN -> 0x7FC0. */
+static uint16_t f32_to_bf16_bits(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0x7FC0;
+    return (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+}
+
+/* Rotary position embedding, rotate-half layout (reading for the fused RoPE):
+ * element i and i + D/2 (i < D/2) turn by the angle of pair i at the row's
+ * position, given as cs[2i] = cos, cs[2i+1] = sin (the caller's table row):
+ *   x'_i       = fl(fl(x_i cos) - fl(x_{i+D/2} sin))
+ *   x'_{i+D/2} = fl(fl(x_{i+D/2} cos) + fl(x_i sin))
+ * one IEEE op each, no FMA contraction. */
+void oracle_rope_f32(float* x, int D, const float* cs) {
+    int half = D / 2;
+    for (int i = 0; i < half; i++) {
+        float c = cs[2 * i], s = cs[2 * i + 1];
+        float a = x[i], b = x[i + half];
+        float ac = a * c, bs = b * s, bc = b * c, as = a * s;
+        x[i] = ac - bs;
+        x[i + half] = bc + as;
+    }
+}
+
 void oracle_rotate_f32(float* x, int D, int b, int normalise) {
     for (int base = 0; base < D; base += b) {
         float* blk = x + base;
@@ -214,12 +243,12 @@ int64_t oracle_append(int mode, int bdr_block, int rotate_v, int num_pages, int 
                       int H, int D, uint8_t* k_pool, uint8_t* v_pool, uint16_t* k_sz,
                       uint16_t* v_sz, const uint16_t* k, const uint16_t* v, int num_tokens,
                       const int32_t* tok_seq, const int32_t* tok_pos, const int32_t* page_table,
-                      int pt_stride, int num_seqs) {
+                      int pt_stride, int num_seqs, const float* rope, int rope_positions) {
     int64_t skipped = 0;
     float* y = (float*)malloc(sizeof(float) * (size_t)D);
     for (int i = 0; i < num_tokens; i++) {
         int s = tok_seq[i], p = tok_pos[i];
-        if (s < 0 || s >= num_seqs || p < 0 || p / page_size >= pt_stride) {
+        if (s < 0 || s >= num_seqs || p < 0 || p / page_size >= pt_stride || (rope && p >= rope_positions)) {
             skipped++;
             continue;
         }
@@ -233,12 +262,20 @@ int64_t oracle_append(int mode, int bdr_block, int rotate_v, int num_pages, int 
             int64_t row = ((int64_t)page * H + h) * page_size + slot;
             for (int kv = 0; kv < 2; kv++) {
                 const uint16_t* src = (kv == 0 ? k : v) + ((int64_t)i * H + h) * D;
+                int rotary = rope && kv == 0; /* RoPE turns the keys only */
                 if (mode == KVQO_BF16) {
                     uint16_t* dst = (uint16_t*)(kv == 0 ? k_pool : v_pool) + row * D;
-                    memcpy(dst, src, sizeof(uint16_t) * (size_t)D);
+                    if (!rotary) {
+                        memcpy(dst, src, sizeof(uint16_t) * (size_t)D);
+                    } else {
+                        for (int e = 0; e < D; e++) y[e] = bf16_bits_to_f32(src[e]);
+                        oracle_rope_f32(y, D, rope + (int64_t)p * D);
+                        for (int e = 0; e < D; e++) dst[e] = f32_to_bf16_bits(y[e]);
+                    }
                     continue;
                 }
                 for (int e = 0; e < D; e++) y[e] = bf16_bits_to_f32(src[e]);
+                if (rotary) oracle_rope_f32(y, D, rope + (int64_t)p * D);
                 int rotate = (mode == KVQO_INT4_BDR) && (kv == 0 || rotate_v);
                 if (rotate) oracle_rotate_f32(y, D, bdr_block, 1);
                 uint8_t* cdst = (kv == 0 ? k_pool : v_pool) + row * (D / 2);
@@ -271,7 +308,7 @@ int64_t oracle_decode(int mode, int bdr_block, int rotate_v, int num_pages, int 
                       int Hq, int D, const void* k_pool, const void* v_pool, const uint16_t* k_sz,
                       const uint16_t* v_sz, const uint16_t* q, const int32_t* seq_lens,
                       const int32_t* page_table, int pt_stride, int batch, const int32_t* rows,
-                      int num_rows, double* out) {
+                      int num_rows, double* out, const float* rope, int rope_positions) {
     int64_t skipped = 0;
     int G = Hq / H;
     int n = rows ? num_rows : batch * Hq;
@@ -282,9 +319,25 @@ int64_t oracle_decode(int mode, int bdr_block, int rotate_v, int num_pages, int 
         int j = rows ? rows[2 * r + 1] : r % Hq;
         int h = j / G;
         for (int e = 0; e < D; e++) qr[e] = (double)bf16_bits_to_f32(q[((int64_t)s * Hq + j) * D + e]);
-        if (mode == KVQO_INT4_BDR) oracle_rotate_f64(qr, D, bdr_block);
         int L = seq_lens[s];
         if (L < 0) L = 0;
+        if (rope && L > 0) {
+            /* the query is the newest token, at position L - 1 (reading); a position outside the
+             * table skips the sequence: zero output */
+            if (L > rope_positions) {
+                skipped += L;
+                for (int e = 0; e < D; e++) out[(int64_t)r * D + e] = 0.0;
+                continue;
+            }
+            const float* cs = rope + (int64_t)(L - 1) * D;
+            for (int i = 0; i < D / 2; i++) {
+                double c = (double)cs[2 * i], sn = (double)cs[2 * i + 1];
+                double a = qr[i], b = qr[i + D / 2];
+                qr[i] = a * c - b * sn;
+                qr[i + D / 2] = b * c + a * sn;
+            }
+        }
+        if (mode == KVQO_INT4_BDR) oracle_rotate_f64(qr, D, bdr_block);
         if (L > pt_stride * page_size) { /* positions beyond the page table */
             skipped += L - pt_stride * page_size;
             L = pt_stride * page_size;
