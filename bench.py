@@ -214,15 +214,16 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples)}
 
 
-def make_cache(w: Workload, mode, b, rv, device):
-    cache = kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0)
+def make_cache(w: Workload, mode, b, rv, device, rope=None):
+    cache = kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0, rope=rope)
     w.run_prefill(cache)
     return cache
 
 
-def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False):
-    """Device-timed steps (CUDA events on the launching stream); per-kernel and per-step means (ms)."""
-    cache = make_cache(w, mode, b, rv, device)
+def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False, rope=None):
+    """Device-timed steps (CUDA events on the launching stream); per-kernel and per-step means (ms).
+    rope: optional (cos, sin) table for the fused rotary embedding."""
+    cache = make_cache(w, mode, b, rv, device, rope)
     ws, _ = cache.workspace(w.dec_B, w.max_len, device)
     out = torch.empty(w.dec_B, w.Hq, 128, dtype=torch.bfloat16, device=device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -490,6 +491,14 @@ def main():
                            "decode_gbs": w.decode_bytes(mode) / (r["decode_ms"] / 1e3) / 1e9,
                            "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3}
         sweep["bdr128_k_over_int4_append"] = sweep["bdr128_k"]["append_tok_per_s"] / sweep["int4"]["append_tok_per_s"]
+        # the same step with the fused rotary embedding (keys turned in the append, q in the decode)
+        tab = synth.rope_table(max(w.dec_lens) + 1).to(device)
+        r = run_variant(w, kvq.KV_INT4_BDR, 128, False, n, 3, device, rope=tab)
+        sweep["bdr128_k_rope"] = {"append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
+                                  "append_gbs": w.append_bytes(kvq.KV_INT4_BDR) / (r["append_ms"] / 1e3) / 1e9,
+                                  "decode_gbs": w.decode_bytes(kvq.KV_INT4_BDR) / (r["decode_ms"] / 1e3) / 1e9,
+                                  "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3,
+                                  "note": "plus the table reads (512 B per appended token, L2-resident)"}
 
     accuracy = None
     if not args.no_accuracy and args.workload in ("batch16", "single256"):

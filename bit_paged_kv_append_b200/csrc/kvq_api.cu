@@ -54,6 +54,7 @@ kv_status kv_create_paged(const kv_desc* d, kv_cache** out) {
     if (!d->k_pool || !d->v_pool || !aligned(d->k_pool, 32) || !aligned(d->v_pool, 32)) return KV_ERR_INVALID;
     if (d->mode != KV_BF16 && (!d->k_sz || !d->v_sz || !aligned(d->k_sz, 16) || !aligned(d->v_sz, 16)))
         return KV_ERR_INVALID;
+    if (d->rope && (d->rope_positions < 1 || !aligned(d->rope, 16))) return KV_ERR_INVALID;
     const int64_t rows = int64_t(d->num_pages) * d->num_kv_heads * d->page_size;
     if (rows >= (int64_t(1) << 32)) return KV_ERR_INVALID;  // slot indices are 32-bit in the kernels
 
@@ -71,6 +72,8 @@ kv_status kv_create_paged(const kv_desc* d, kv_cache** out) {
     c->g.v_pool = d->v_pool;
     c->g.k_sz = static_cast<uint32_t*>(d->mode == KV_BF16 ? nullptr : d->k_sz);
     c->g.v_sz = static_cast<uint32_t*>(d->mode == KV_BF16 ? nullptr : d->v_sz);
+    c->g.rope = d->rope;
+    c->g.rope_positions = d->rope ? d->rope_positions : 0;
     if (cudaGetDevice(&c->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess ||
         cudaMalloc(&c->err_dev, sizeof(int)) != cudaSuccess) {

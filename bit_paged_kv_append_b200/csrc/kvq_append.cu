@@ -44,7 +44,8 @@ constexpr int kHalfBytes = kRows * 128;      // one 128-byte half-row per row
 constexpr int kStageBytes = 2 * kHalfBytes;  // 56 KiB (a multiple of 1 KiB: swizzle atoms stay aligned)
 constexpr int kMaxTileTokens = kRows;        // H == 1
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kStages) * kStageBytes +
-                              2 * size_t(kMaxTileTokens) * sizeof(int2) + 2 * kStages * sizeof(uint64_t);
+                              2 * size_t(kMaxTileTokens) * (sizeof(int2) + sizeof(int)) +
+                              2 * kStages * sizeof(uint64_t);
 
 // Magic constant 1.5 * 2^23: for |v| < 2^22, the fp32 sum v + kMagic (rounded to
 // nearest even) carries rint_even(v) in its low mantissa bits.
@@ -221,11 +222,59 @@ __device__ __forceinline__ void quantise_store(const float2 (&R)[64], uint8_t* c
     *sz_dst = uint32_t(__half_as_ushort(sh)) | (uint32_t(__half_as_ushort(zh)) << 16);
 }
 
-template <bool ROT, int BLK>
-__device__ __forceinline__ void process_row(const uint8_t* stage, int row, float r_b, uint8_t* cdst,
-                                            uint32_t* sdst) {
+// Rotary embedding of one row, rotate-half pairs: R[i] = (x_i, x_{i+64}) turns by the
+// angle of pair i at the token's position, cs = that position's (cos, sin) table row:
+// x_i' = fl(fl(x_i c) - fl(x_{i+64} s)), x_{i+64}' = fl(fl(x_{i+64} c) + fl(x_i s)),
+// scalar IEEE ops (never contracted).
+__device__ __forceinline__ void rope_row(float2 (&R)[64], const float* cs) {
+    const float4* t = reinterpret_cast<const float4*>(cs);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const float4 w = __ldg(t + j);  // pairs 2j and 2j + 1: (cos, sin, cos, sin)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float c = e ? w.z : w.x, s = e ? w.w : w.y;
+            const float x = R[2 * j + e].x, y = R[2 * j + e].y;
+            R[2 * j + e] = make_float2(__fsub_rn(__fmul_rn(x, c), __fmul_rn(y, s)),
+                                       __fadd_rn(__fmul_rn(y, c), __fmul_rn(x, s)));
+        }
+    }
+}
+
+// fp32 -> bf16 bits, round to nearest even; NaN -> 0x7FC0
+__device__ __forceinline__ uint32_t bf16_rn_bits(float f) {
+    const uint32_t u = __float_as_uint(f);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0x7FC0u;
+    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+}
+
+// BF16 cache with RoPE: the turned key row, rounded to bf16, into the pool row.
+__device__ __forceinline__ void copy_row_rope(const uint8_t* stage, int row, const float* cs, uint8_t* dst) {
     float2 R[64];
     load_row(stage, row, R);
+    rope_row(R, cs);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // 16 elements (32 bytes) per store
+            uint32_t w[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int i = 16 * q + 2 * k;
+                const float a = half ? R[i].y : R[i].x, b = half ? R[i + 1].y : R[i + 1].x;
+                w[k] = bf16_rn_bits(a) | (bf16_rn_bits(b) << 16);
+            }
+            st_global_v8(dst + half * 128 + q * 32, w);
+        }
+    }
+}
+
+template <bool ROT, int BLK>
+__device__ __forceinline__ void process_row(const uint8_t* stage, int row, float r_b, const float* cs,
+                                            uint8_t* cdst, uint32_t* sdst) {
+    float2 R[64];
+    load_row(stage, row, R);
+    if (cs) rope_row(R, cs);
     if (ROT) rotate_row<BLK>(R, r_b);
     quantise_store(R, cdst, sdst);
 }
@@ -247,14 +296,15 @@ __device__ __forceinline__ void copy_row(const uint8_t* stage, int row, uint8_t*
     }
 }
 
-template <int MODE, int BLK, bool ROTV>
+template <int MODE, int BLK, bool ROTV, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     append_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
     int2* meta = reinterpret_cast<int2*>(smem + kStages * kStageBytes);  // [tile parity][tile token] = (page, slot)
-    uint64_t* full = reinterpret_cast<uint64_t*>(meta + 2 * kMaxTileTokens);
+    int* mpos = reinterpret_cast<int*>(meta + 2 * kMaxTileTokens);       // [tile parity][tile token] = position
+    uint64_t* full = reinterpret_cast<uint64_t*>(mpos + 2 * kMaxTileTokens);
     uint64_t* empty = full + kStages;
 
     const int tid = threadIdx.x;
@@ -314,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // the meta slot of tile n was last read for tile n - 2, whose stages the waits above freed
             int2* mt = meta + (n & 1) * kMaxTileTokens;
+            int* mp = mpos + (n & 1) * kMaxTileTokens;
 #pragma unroll
             for (int r = 0; r < kPerLane; ++r) {
                 const int tt = lane + 32 * r;
@@ -322,7 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     int2 m = make_int2(-1, 0);
                     if (t < p.a.num_tokens) {
                         const int sid = sq[r], pos = po[r];
-                        bool ok = sid >= 0 && sid < p.a.num_seqs && pos >= 0 && pos / p.g.page_size < p.a.pt_stride;
+                        bool ok = sid >= 0 && sid < p.a.num_seqs && pos >= 0 && pos / p.g.page_size < p.a.pt_stride &&
+                                  (!ROPE || pos < p.g.rope_positions);
                         if (ok) {
                             const int page = __ldg(p.a.page_table + int64_t(sid) * p.a.pt_stride + pos / p.g.page_size);
                             ok = page >= 0 && page < p.g.num_pages;
@@ -331,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) flag_error(p.err, kErrOOB);
                     }
                     mt[tt] = m;
+                    if (ROPE) mp[tt] = po[r];
                 }
             }
             __syncwarp();
@@ -360,18 +413,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return;
             }
             if (kv == 0) m = meta[(n & 1) * kMaxTileTokens + tt];
+            // key rows turn at the token's position (the position was checked by the producer)
+            const float* cs = (ROPE && kv == 0 && m.x >= 0)
+                                  ? p.g.rope + int64_t(mpos[(n & 1) * kMaxTileTokens + tt]) * kHeadDim
+                                  : nullptr;
             const int t = tile * TT + tt;
             if (t < p.a.num_tokens && m.x >= 0) {
                 const uint8_t* stage = stages + e * kStageBytes;
                 const int64_t row = (int64_t(m.x) * H + h) * p.g.page_size + m.y;
                 if (MODE == 0) {
                     uint8_t* dst = static_cast<uint8_t*>(kv ? p.g.v_pool : p.g.k_pool) + row * 256;
-                    copy_row(stage, tid, dst);
+                    if (ROPE && cs)
+                        copy_row_rope(stage, tid, cs, dst);
+                    else
+                        copy_row(stage, tid, dst);
                 } else {
                     uint8_t* cdst = static_cast<uint8_t*>(kv ? p.g.v_pool : p.g.k_pool) + row * 64;
                     uint32_t* sdst = (kv ? p.g.v_sz : p.g.k_sz) + row;
-                    if (kv == 0) process_row<MODE == 2, BLK>(stage, tid, p.r_b, cdst, sdst);
-                    else process_row<MODE == 2 && ROTV, BLK>(stage, tid, p.r_b, cdst, sdst);
+                    if (kv == 0) process_row<MODE == 2, BLK>(stage, tid, p.r_b, ROPE ? cs : nullptr, cdst, sdst);
+                    else process_row<MODE == 2 && ROTV, BLK>(stage, tid, p.r_b, nullptr, cdst, sdst);
                 }
             }
             __syncwarp();
@@ -406,9 +466,9 @@ bool make_row_map(CUtensorMap* map, const void* base, int64_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int BLK, bool ROTV>
-cudaError_t launch_t(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
-    auto kern = append_kernel<MODE, BLK, ROTV>;
+template <int MODE, int BLK, bool ROTV, bool ROPE>
+cudaError_t launch_r(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
+    auto kern = append_kernel<MODE, BLK, ROTV, ROPE>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
@@ -416,6 +476,12 @@ cudaError_t launch_t(const CUtensorMap& km, const CUtensorMap& vm, const Params&
         attr_set = true;
     }
     return launch_overlapped(kern, dim3(grid), dim3(kThreads), kSmemBytes, s, km, vm, p);
+}
+
+template <int MODE, int BLK, bool ROTV>
+cudaError_t launch_t(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
+    return p.g.rope ? launch_r<MODE, BLK, ROTV, true>(km, vm, p, grid, s)
+                    : launch_r<MODE, BLK, ROTV, false>(km, vm, p, grid, s);
 }
 
 }  // namespace

@@ -77,8 +77,27 @@ __global__ void __launch_bounds__(kThreads) bf16_split_kernel(Params p) {
     const int64_t out_row0 = partial_row(p, s, k, h * G);
 
     const uint16_t* q = static_cast<const uint16_t*>(p.a.q) + (int64_t(s) * Hq + h * G) * kHeadDim;
+    if (p.g.rope) {  // fused rotary embedding at position seq_len - 1: pairs (i, i + 64)
 #pragma unroll
-    for (int g = 0; g < G; ++g) sm.qs[g][tid] = __uint_as_float(uint32_t(q[g * kHeadDim + tid]) << 16) * p.qscale;
+        for (int g = 0; g < G; ++g) sm.qs[g][tid] = __uint_as_float(uint32_t(q[g * kHeadDim + tid]) << 16);
+        __syncthreads();
+        const int pos = __ldg(p.a.seq_lens + s) - 1;
+        const int i = tid & 63;
+        const float c = __ldg(p.g.rope + int64_t(pos) * kHeadDim + 2 * i);
+        const float sn = __ldg(p.g.rope + int64_t(pos) * kHeadDim + 2 * i + 1);
+        float turned[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float own = sm.qs[g][tid], other = sm.qs[g][tid ^ 64];
+            turned[g] = tid < 64 ? fmaf(own, c, -other * sn) : fmaf(own, c, other * sn);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int g = 0; g < G; ++g) sm.qs[g][tid] = turned[g] * p.qscale;
+    } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g) sm.qs[g][tid] = __uint_as_float(uint32_t(q[g * kHeadDim + tid]) << 16) * p.qscale;
+    }
     __syncthreads();
 
     float m[G], lsum[G], o[G][4];

@@ -48,9 +48,11 @@ __host__ __device__ constexpr int dpos(int j, int k) {
 }
 
 #ifdef __CUDACC__
-// Cached length of sequence s, clamped to what the page table and the bound allow.
+// Cached length of sequence s, clamped to what the page table and the bound allow; 0 when
+// the fused rotary embedding has no table row for the query's position L - 1.
 __device__ __forceinline__ int decode_len(const DecodeParams& p, int s) {
     const int L = __ldg(p.a.seq_lens + s);
+    if (p.g.rope && L > p.g.rope_positions) return 0;
     const int cap = min(p.a.pt_stride * p.g.page_size, p.a.max_seq_len);
     return L < 0 ? 0 : (L > cap ? cap : L);
 }

@@ -276,14 +276,29 @@ struct ChunkStream {
     }
 };
 
-// Query row qrow (bf16, 128 dims) as q H_blk * log2(e)/sqrt(D): lane holds dims 4 lane .. 4 lane + 3.
-__device__ __forceinline__ void load_q_rotated(const DecodeParams& p, int64_t qrow, int lane, float (&x)[4]) {
+// Query row qrow (bf16, 128 dims) of sequence s as q H_blk * log2(e)/sqrt(D), after the fused
+// rotary embedding at position seq_len - 1 when a table is set: lane holds dims 4 lane ..
+// 4 lane + 3, and lanes l, l ^ 16 hold the rotate-half pairs (i, i + 64).
+__device__ __forceinline__ void load_q_rotated(const DecodeParams& p, int s, int64_t qrow, int lane,
+                                               float (&x)[4]) {
     const uint2 raw =
         __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.a.q) + qrow * kHeadDim) + lane);
     x[0] = __uint_as_float(raw.x << 16);
     x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
     x[2] = __uint_as_float(raw.y << 16);
     x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    if (p.g.rope) {  // the CTA only runs when the position has a table row (decode_len)
+        const int pos = __ldg(p.a.seq_lens + s) - 1;
+        const float4* cs = reinterpret_cast<const float4*>(p.g.rope + int64_t(pos) * kHeadDim) + 2 * (lane & 15);
+        const float4 c01 = __ldg(cs), c23 = __ldg(cs + 1);  // pairs 4 (lane & 15) .. + 3: (cos, sin) each
+        const float c[4] = {c01.x, c01.z, c23.x, c23.z}, sn[4] = {c01.y, c01.w, c23.y, c23.w};
+        const bool upper = lane >= 16;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float other = __shfl_xor_sync(kFull, x[e], 16);
+            x[e] = upper ? fmaf(x[e], c[e], other * sn[e]) : fmaf(x[e], c[e], -other * sn[e]);
+        }
+    }
     float sc = p.qscale;
     if (p.g.mode == 2) {
         const int b = p.g.bdr_block;
@@ -446,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
     // 0..7 lo, rows 8..15 zero.
     for (int row = warp; row < G; row += kWarps) {
         float x[4];
-        load_q_rotated(p, int64_t(s) * p.g.Hq + h * G + row, lane, x);
+        load_q_rotated(p, s, int64_t(s) * p.g.Hq + h * G + row, lane, x);
         float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
@@ -663,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
     // 2 head: lo.
     for (int row = warp; row < G; row += kWarps) {
         float x[4];
-        load_q_rotated(p, int64_t(s) * p.g.Hq + h * G + row, lane, x);
+        load_q_rotated(p, s, int64_t(s) * p.g.Hq + h * G + row, lane, x);
         float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));

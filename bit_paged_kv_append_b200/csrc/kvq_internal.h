@@ -15,6 +15,8 @@ struct CacheGeom {
     void* v_pool;
     uint32_t* k_sz;  // (scale, zero) fp16 pairs as one 32-bit word, scale in the low half
     uint32_t* v_sz;
+    const float* rope;   // (cos, sin) [rope_positions][D/2][2], or nullptr
+    int rope_positions;
 };
 
 struct AppendArgs {

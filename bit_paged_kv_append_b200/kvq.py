@@ -35,7 +35,8 @@ class kv_desc(ctypes.Structure):
     _fields_ = [("num_pages", ctypes.c_int), ("page_size", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
                 ("num_q_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("mode", ctypes.c_int),
                 ("bdr_block", ctypes.c_int), ("rotate_v", ctypes.c_int), ("k_pool", ctypes.c_void_p),
-                ("v_pool", ctypes.c_void_p), ("k_sz", ctypes.c_void_p), ("v_sz", ctypes.c_void_p)]
+                ("v_pool", ctypes.c_void_p), ("k_sz", ctypes.c_void_p), ("v_sz", ctypes.c_void_p),
+                ("rope", ctypes.c_void_p), ("rope_positions", ctypes.c_int)]
 
 
 _lib = None
@@ -99,10 +100,12 @@ def _check(status: int, what: str):
 
 
 def kv_create_paged(num_pages, page_size, num_kv_heads, num_q_heads, head_dim, mode, bdr_block, rotate_v,
-                    k_pool, v_pool, k_sz=None, v_sz=None) -> int:
-    """Returns the opaque handle (an integer address); release it with kv_free."""
+                    k_pool, v_pool, k_sz=None, v_sz=None, rope=None) -> int:
+    """Returns the opaque handle (an integer address); release it with kv_free.  rope: optional
+    device float32 [positions, head_dim/2, 2] (cos, sin) table (fused rotary embedding)."""
     d = kv_desc(num_pages, page_size, num_kv_heads, num_q_heads, head_dim, mode, bdr_block, int(bool(rotate_v)),
-                _ptr(k_pool), _ptr(v_pool), _ptr(k_sz), _ptr(v_sz))
+                _ptr(k_pool), _ptr(v_pool), _ptr(k_sz), _ptr(v_sz), _ptr(rope),
+                int(rope.shape[0]) if rope is not None else 0)
     h = ctypes.c_void_p()
     _check(load().kv_create_paged(ctypes.byref(d), ctypes.byref(h)), "kv_create_paged")
     return h.value
@@ -173,14 +176,15 @@ class PagedKVCache:
     """Owns one handle over caller-provided (or freshly allocated) pools."""
 
     def __init__(self, num_pages, page_size, num_kv_heads, num_q_heads, mode, bdr_block=128, rotate_v=False,
-                 pools=None, device="cuda", fill=None):
+                 pools=None, device="cuda", fill=None, rope=None):
         self.mode, self.bdr_block, self.rotate_v = mode, bdr_block, bool(rotate_v)
+        self.rope = rope  # kept alive with the handle
         self.num_pages, self.page_size = num_pages, page_size
         self.num_kv_heads, self.num_q_heads = num_kv_heads, num_q_heads
         self.k_pool, self.v_pool, self.k_sz, self.v_sz = pools or alloc_pools(num_pages, page_size, num_kv_heads,
                                                                                mode, device, fill)
         self.handle = kv_create_paged(num_pages, page_size, num_kv_heads, num_q_heads, HEAD_DIM, mode, bdr_block,
-                                      rotate_v, self.k_pool, self.v_pool, self.k_sz, self.v_sz)
+                                      rotate_v, self.k_pool, self.v_pool, self.k_sz, self.v_sz, rope)
 
     def append(self, k, v, tok_seq, tok_pos, page_table, stream=None):
         kv_append_quant(self.handle, k, v, k.shape[0], tok_seq, tok_pos, page_table, page_table.shape[1],

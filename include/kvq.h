@@ -92,6 +92,16 @@ typedef struct {
     void* v_pool;
     void* k_sz;       /* device fp16x2 scale/zero arrays (INT4 modes), 16-byte aligned; NULL for BF16 */
     void* v_sz;
+    /* Optional fused rotary embedding: NULL = off.  Else a device float32 table
+     * [rope_positions][head_dim/2][2] (cos, sin) of each position's angle for the
+     * rotate-half pairs (i, i + head_dim/2), 16-byte aligned, owned by the caller.
+     * kv_append_quant turns each key row at its tok_pos (fp32, before the block
+     * rotation; BF16 pages store the turned row rounded to nearest even);
+     * kv_decode_attn turns q at position seq_len - 1 (the newest token).  A
+     * position outside the table skips the token (append) or the sequence (decode:
+     * zero output), flagged KV_ERR_OOB. */
+    const float* rope;
+    int rope_positions; /* rows of the table (>= 1 when rope is set) */
 } kv_desc;
 
 typedef struct kv_cache kv_cache; /* opaque host handle */

@@ -63,6 +63,8 @@ def _desc(**kw):
     (dict(k_pool=0), kvq.KV_ERR_INVALID),
     (dict(v_pool=0x2010), kvq.KV_ERR_INVALID),  # not 32-byte aligned
     (dict(k_sz=0), kvq.KV_ERR_INVALID),
+    (dict(rope=0x5000, rope_positions=0), kvq.KV_ERR_INVALID),  # a table needs >= 1 row
+    (dict(rope=0x5004, rope_positions=8), kvq.KV_ERR_INVALID),  # not 16-byte aligned
 ])
 def test_create_rejects_bad_descriptors(kw, status):
     lib = kvq.load()
