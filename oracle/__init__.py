@@ -57,12 +57,14 @@ def _load():
         lib.oracle_rotate_f64.argtypes = [P, ctypes.c_int, ctypes.c_int]
         lib.oracle_quant_row.argtypes = [P, ctypes.c_int, P, P]
         lib.oracle_quant_rows.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P]
+        lib.oracle_quant_row_bits.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P]
+        lib.oracle_quant_rows_bits.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
         lib.oracle_append.restype = i64
         lib.oracle_append.argtypes = [ctypes.c_int] * 7 + [P] * 6 + [ctypes.c_int, P, P, P, ctypes.c_int,
-                                                                     ctypes.c_int, P, ctypes.c_int]
+                                                                     ctypes.c_int, P, ctypes.c_int, ctypes.c_int]
         lib.oracle_decode.restype = i64
         lib.oracle_decode.argtypes = [ctypes.c_int] * 8 + [P] * 7 + [ctypes.c_int, ctypes.c_int, P,
-                                                                     ctypes.c_int, P, P, ctypes.c_int]
+                                                                     ctypes.c_int, P, P, ctypes.c_int, ctypes.c_int]
         lib.oracle_rope_f32.argtypes = [P, ctypes.c_int, P]
         _lib = lib
     return _lib
@@ -105,32 +107,33 @@ def rotate_f64(x: np.ndarray, b: int) -> np.ndarray:
     return x
 
 
-def quant_row(y: np.ndarray):
-    """Token-wise asymmetric INT4 of one fp32 row -> (packed codes uint8[D/2], (scale, zero) fp16 bits)."""
+def quant_row(y: np.ndarray, bits: int = 4):
+    """Token-wise asymmetric INT4 (bits = 4) or INT2 (bits = 2) of one fp32 row -> (packed codes
+    uint8[D * bits / 8], (scale, zero) fp16 bits)."""
     y = np.ascontiguousarray(y, dtype=np.float32)
     D = y.shape[0]
-    codes = np.empty(D // 2, dtype=np.uint8)
+    codes = np.empty(D * bits // 8, dtype=np.uint8)
     sz = np.empty(2, dtype=np.uint16)
-    _load().oracle_quant_row(_ptr(y), D, _ptr(codes), _ptr(sz))
+    _load().oracle_quant_row_bits(_ptr(y), D, bits, _ptr(codes), _ptr(sz))
     return codes, sz
 
 
-def quant_rows(x_bf16_bits: np.ndarray, b: int):
-    """Rotate (block b; b == 0: none) and quantise bf16 rows [..., D] -> (codes [..., D/2], sz [..., 2])."""
+def quant_rows(x_bf16_bits: np.ndarray, b: int, bits: int = 4):
+    """Rotate (block b; b == 0: none) and quantise bf16 rows [..., D] -> (codes [..., D*bits/8], sz [..., 2])."""
     x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
     D = x.shape[-1]
     n = x.size // D
-    codes = np.empty(x.shape[:-1] + (D // 2,), dtype=np.uint8)
+    codes = np.empty(x.shape[:-1] + (D * bits // 8,), dtype=np.uint8)
     sz = np.empty(x.shape[:-1] + (2,), dtype=np.uint16)
-    _load().oracle_quant_rows(_ptr(x), n, D, b, _ptr(codes), _ptr(sz))
+    _load().oracle_quant_rows_bits(_ptr(x), n, D, b, bits, _ptr(codes), _ptr(sz))
     return codes, sz
 
 
-def unpack_codes(codes: np.ndarray) -> np.ndarray:
-    """Packed bytes [..., D/2] -> codes [..., D] (low nibble = even element)."""
-    lo = codes & 15
-    hi = codes >> 4
-    return np.stack([lo, hi], axis=-1).reshape(codes.shape[:-1] + (codes.shape[-1] * 2,))
+def unpack_codes(codes: np.ndarray, bits: int = 4) -> np.ndarray:
+    """Packed bytes [..., D*bits/8] -> codes [..., D] (code k of a byte in bits k*bits ..)."""
+    per = 8 // bits
+    parts = [(codes >> (bits * k)) & ((1 << bits) - 1) for k in range(per)]
+    return np.stack(parts, axis=-1).reshape(codes.shape[:-1] + (codes.shape[-1] * per,))
 
 
 def _rope_args(rope):
@@ -150,7 +153,7 @@ def rope_f32(x: np.ndarray, cs: np.ndarray) -> np.ndarray:
 
 
 def append(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz, k_bits, v_bits,
-           tok_seq, tok_pos, page_table, rope=None) -> int:
+           tok_seq, tok_pos, page_table, rope=None, code_bits: int = 4) -> int:
     """Append tokens into the pools in place (numpy arrays); returns the skipped-token count.
 
     Pools: INT4 uint8 [P, H, ps, D/2] (+ sz uint16 [P, H, ps, 2]); BF16 uint16 [P, H, ps, D].
@@ -167,11 +170,11 @@ def append(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz
     return int(_load().oracle_append(mode, bdr_block, int(rotate_v), P, ps, H, D, _ptr(k_pool), _ptr(v_pool),
                                      _ptr(k_sz), _ptr(v_sz), _ptr(np.ascontiguousarray(k_bits)),
                                      _ptr(np.ascontiguousarray(v_bits)), T, _ptr(ts), _ptr(tp), _ptr(pt),
-                                     pt.shape[1], pt.shape[0], rp, rn))
+                                     pt.shape[1], pt.shape[0], rp, rn, int(code_bits)))
 
 
 def decode(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz, q_bits, seq_lens,
-           page_table, num_kv_heads: int, rows=None, rope=None):
+           page_table, num_kv_heads: int, rows=None, rope=None, code_bits: int = 4):
     """Paged GQA decode attention in float64.
 
     q_bits: bf16 bits uint16 [B, Hq, D].  rows: optional int array [(seq, qhead), ...]; when None all
@@ -193,7 +196,8 @@ def decode(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz
     keep, rp, rn = _rope_args(rope)
     skipped = _load().oracle_decode(mode, bdr_block, int(rotate_v), P, ps, num_kv_heads, Hq, D, _ptr(k_pool),
                                     _ptr(v_pool), _ptr(k_sz), _ptr(v_sz), _ptr(np.ascontiguousarray(q_bits)),
-                                    _ptr(sl), _ptr(pt), pt.shape[1], B, _ptr(rws), n, _ptr(out), rp, rn)
+                                    _ptr(sl), _ptr(pt), pt.shape[1], B, _ptr(rws), n, _ptr(out), rp, rn,
+                                    int(code_bits))
     if rows is None:
         out = out.reshape(B, Hq, D)
     return out, int(skipped)

@@ -47,6 +47,8 @@
  *     fp32 before the rounding to an integer).  A row holding a NaN has NaN
  *     min and max: scale = zero = fp16 quiet NaN 0x7E00 and every code 0.
  *     Dequantised value = code * scale + zero.
+ *  2-bit variant (optional): the same quantiser with range/3, codes 0..3, four
+ *     codes per byte, code k of a byte in bits 2k and 2k+1.
  *  Fused RoPE (optional): a caller-given table of (cos, sin) per position and
  *     rotate-half pair turns the keys (fp32, before the block rotation; BF16
  *     pages store the turned row rounded to bf16) and the query, at position
@@ -177,14 +179,19 @@ void oracle_rotate_f64(double* x, int D, int b) {
 
 /* ---- token-wise asymmetric INT4 (C1, [ABS], [WIS3]; readings R3-R5) ------ */
 
-/* Quantise one (already rotated) row y[0..D) into D/2 packed bytes and an
- * (scale, zero) fp16 pair. */
-void oracle_quant_row(const float* y, int D, uint8_t* codes, uint16_t* scale_zero) {
+/* Quantise one (already rotated) row y[0..D) into D*bits/8 packed bytes and an
+ * (scale, zero) fp16 pair: bits = 4 (codes 0..15, two per byte) or 2 (codes
+ * 0..3, four per byte; reading for the 2-bit variant: the same token-wise
+ * asymmetric quantiser with range/3, code k of a byte in bits 2k, 2k+1). */
+void oracle_quant_row_bits(const float* y, int D, int bits, uint8_t* codes, uint16_t* scale_zero) {
+    const int levels = (1 << bits) - 1;
+    const int per_byte = 8 / bits;
+    const int nbytes = D / per_byte;
     /* a NaN anywhere makes the row's min and max NaN (reading): scale and zero are the
      * fp16 quiet NaN 0x7E00 and every code is 0 */
     for (int i = 0; i < D; i++) {
         if (y[i] != y[i]) {
-            for (int j = 0; j < D / 2; j++) codes[j] = 0;
+            for (int j = 0; j < nbytes; j++) codes[j] = 0;
             scale_zero[0] = scale_zero[1] = 0x7E00;
             return;
         }
@@ -197,41 +204,45 @@ void oracle_quant_row(const float* y, int D, uint8_t* codes, uint16_t* scale_zer
     mn = mn + 0.0f; /* -0 + +0 = +0: signed zeros made canonical */
     mx = mx + 0.0f;
     float range = mx - mn;
-    float s32 = range / 15.0f;
+    float s32 = range / (float)levels;
     uint16_t scale_h = f32_to_f16_bits(s32);
     uint16_t zero_h = f32_to_f16_bits(mn);
     float scale = f16_bits_to_f32(scale_h);
     float zero = f16_bits_to_f32(zero_h);
     float inv = (scale > 0.0f) ? 1.0f / scale : 0.0f;
-    for (int j = 0; j < D / 2; j++) {
-        int c[2];
-        for (int e = 0; e < 2; e++) {
-            float t = y[2 * j + e] - zero;
-            /* the quotient t * inv is rounded to an integer from its exact value: the
-             * product of two floats is exact in double (24 + 24 < 53 significant bits) */
-            double v = (double)t * (double)inv;
-            double r = rint(v); /* default rounding mode: nearest, ties to even */
-            int code;
-            if (!(r > 0.0)) code = 0; /* also NaN */
-            else if (r > 15.0) code = 15;
-            else code = (int)r;
-            c[e] = code;
-        }
-        codes[j] = (uint8_t)(c[0] | (c[1] << 4));
+    for (int j = 0; j < nbytes; j++) codes[j] = 0;
+    for (int e = 0; e < D; e++) {
+        float t = y[e] - zero;
+        /* the quotient t * inv is rounded to an integer from its exact value: the
+         * product of two floats is exact in double (24 + 24 < 53 significant bits) */
+        double v = (double)t * (double)inv;
+        double r = rint(v); /* default rounding mode: nearest, ties to even */
+        int code;
+        if (!(r > 0.0)) code = 0; /* also NaN */
+        else if (r > (double)levels) code = levels;
+        else code = (int)r;
+        codes[e / per_byte] |= (uint8_t)(code << (bits * (e % per_byte)));
     }
     scale_zero[0] = scale_h;
     scale_zero[1] = zero_h;
 }
 
-/* Rotate (block b, or none when b == 0) and quantise n rows of bf16 input. */
-void oracle_quant_rows(const uint16_t* x, int64_t n, int D, int b, uint8_t* codes, uint16_t* sz) {
+void oracle_quant_row(const float* y, int D, uint8_t* codes, uint16_t* scale_zero) {
+    oracle_quant_row_bits(y, D, 4, codes, scale_zero);
+}
+
+void oracle_quant_rows_bits(const uint16_t* x, int64_t n, int D, int b, int bits, uint8_t* codes, uint16_t* sz) {
     float* y = (float*)malloc(sizeof(float) * (size_t)D);
     for (int64_t r = 0; r < n; r++) {
         for (int i = 0; i < D; i++) y[i] = bf16_bits_to_f32(x[r * D + i]);
         if (b > 0) oracle_rotate_f32(y, D, b, 1);
-        oracle_quant_row(y, D, codes + r * (D / 2), sz + r * 2);
+        oracle_quant_row_bits(y, D, bits, codes + r * (D * bits / 8), sz + r * 2);
     }
     free(y);
+}
+
+void oracle_quant_rows(const uint16_t* x, int64_t n, int D, int b, uint8_t* codes, uint16_t* sz) {
+    oracle_quant_rows_bits(x, n, D, b, 4, codes, sz);
 }
 
 /* ---- append into the paged cache (C3, C5, C6; reading R6, R8) ------------ */
@@ -243,9 +254,10 @@ int64_t oracle_append(int mode, int bdr_block, int rotate_v, int num_pages, int 
                       int H, int D, uint8_t* k_pool, uint8_t* v_pool, uint16_t* k_sz,
                       uint16_t* v_sz, const uint16_t* k, const uint16_t* v, int num_tokens,
                       const int32_t* tok_seq, const int32_t* tok_pos, const int32_t* page_table,
-                      int pt_stride, int num_seqs, const float* rope, int rope_positions) {
+                      int pt_stride, int num_seqs, const float* rope, int rope_positions, int bits) {
     int64_t skipped = 0;
     float* y = (float*)malloc(sizeof(float) * (size_t)D);
+    const int row_bytes = D * bits / 8;
     for (int i = 0; i < num_tokens; i++) {
         int s = tok_seq[i], p = tok_pos[i];
         if (s < 0 || s >= num_seqs || p < 0 || p / page_size >= pt_stride || (rope && p >= rope_positions)) {
@@ -278,9 +290,9 @@ int64_t oracle_append(int mode, int bdr_block, int rotate_v, int num_pages, int 
                 if (rotary) oracle_rope_f32(y, D, rope + (int64_t)p * D);
                 int rotate = (mode == KVQO_INT4_BDR) && (kv == 0 || rotate_v);
                 if (rotate) oracle_rotate_f32(y, D, bdr_block, 1);
-                uint8_t* cdst = (kv == 0 ? k_pool : v_pool) + row * (D / 2);
+                uint8_t* cdst = (kv == 0 ? k_pool : v_pool) + row * row_bytes;
                 uint16_t* sdst = (kv == 0 ? k_sz : v_sz) + row * 2;
-                oracle_quant_row(y, D, cdst, sdst);
+                oracle_quant_row_bits(y, D, bits, cdst, sdst);
             }
         }
     }
@@ -291,10 +303,11 @@ int64_t oracle_append(int mode, int bdr_block, int rotate_v, int num_pages, int 
 /* ---- decode attention over the paged cache (C4, C7; readings R6-R8) ------ */
 
 /* Dequantised element e of the cached row (page, h, slot), as float64. */
-static double cached_value(int mode, const void* pool, const uint16_t* sz, int64_t row, int D, int e) {
+static double cached_value(int mode, int bits, const void* pool, const uint16_t* sz, int64_t row, int D, int e) {
     if (mode == KVQO_BF16) return (double)bf16_bits_to_f32(((const uint16_t*)pool)[row * D + e]);
-    uint8_t byte = ((const uint8_t*)pool)[row * (D / 2) + e / 2];
-    int code = (e % 2 == 0) ? (byte & 15) : (byte >> 4);
+    const int per_byte = 8 / bits;
+    uint8_t byte = ((const uint8_t*)pool)[row * (D / per_byte) + e / per_byte];
+    int code = (byte >> (bits * (e % per_byte))) & ((1 << bits) - 1);
     double scale = (double)f16_bits_to_f32(sz[row * 2 + 0]);
     double zero = (double)f16_bits_to_f32(sz[row * 2 + 1]);
     return (double)code * scale + zero;
@@ -308,7 +321,7 @@ int64_t oracle_decode(int mode, int bdr_block, int rotate_v, int num_pages, int 
                       int Hq, int D, const void* k_pool, const void* v_pool, const uint16_t* k_sz,
                       const uint16_t* v_sz, const uint16_t* q, const int32_t* seq_lens,
                       const int32_t* page_table, int pt_stride, int batch, const int32_t* rows,
-                      int num_rows, double* out, const float* rope, int rope_positions) {
+                      int num_rows, double* out, const float* rope, int rope_positions, int bits) {
     int64_t skipped = 0;
     int G = Hq / H;
     int n = rows ? num_rows : batch * Hq;
@@ -355,7 +368,7 @@ int64_t oracle_decode(int mode, int bdr_block, int rotate_v, int num_pages, int 
             int64_t row = ((int64_t)page * H + h) * page_size + t % page_size;
             rowid[t] = row;
             double dot = 0.0;
-            for (int e = 0; e < D; e++) dot += qr[e] * cached_value(mode, k_pool, k_sz, row, D, e);
+            for (int e = 0; e < D; e++) dot += qr[e] * cached_value(mode, bits, k_pool, k_sz, row, D, e);
             z[t] = dot / sqrt((double)D);
             if (z[t] > zmax) zmax = z[t];
         }
@@ -365,7 +378,7 @@ int64_t oracle_decode(int mode, int bdr_block, int rotate_v, int num_pages, int 
             if (rowid[t] < 0) continue;
             double p = exp(z[t] - zmax);
             l += p;
-            for (int e = 0; e < D; e++) o[e] += p * cached_value(mode, v_pool, v_sz, rowid[t], D, e);
+            for (int e = 0; e < D; e++) o[e] += p * cached_value(mode, bits, v_pool, v_sz, rowid[t], D, e);
         }
         if (l > 0.0)
             for (int e = 0; e < D; e++) o[e] /= l;
