@@ -214,16 +214,17 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples)}
 
 
-def make_cache(w: Workload, mode, b, rv, device, rope=None):
-    cache = kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0, rope=rope)
+def make_cache(w: Workload, mode, b, rv, device, rope=None, code_bits=4):
+    cache = kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0, rope=rope,
+                             code_bits=code_bits)
     w.run_prefill(cache)
     return cache
 
 
-def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False, rope=None):
+def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False, rope=None, code_bits=4):
     """Device-timed steps (CUDA events on the launching stream); per-kernel and per-step means (ms).
-    rope: optional (cos, sin) table for the fused rotary embedding."""
-    cache = make_cache(w, mode, b, rv, device, rope)
+    rope: optional (cos, sin) table for the fused rotary embedding; code_bits: 4 or 2."""
+    cache = make_cache(w, mode, b, rv, device, rope, code_bits)
     ws, _ = cache.workspace(w.dec_B, w.max_len, device)
     out = torch.empty(w.dec_B, w.Hq, 128, dtype=torch.bfloat16, device=device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -308,8 +309,10 @@ def accuracy_study(w: Workload, device):
     ref = exact_attention(k, v, w.q, w.dec_lens, w.H, w.Hq)
     den = np.maximum(np.abs(ref).max(axis=-1), 1e-30)
     res = {}
-    for name, mode, b, rv in VARIANTS:
-        cache = kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0)
+    two_bit = [("int2", kvq.KV_INT4, 0, False, 2), ("bdr128_k_int2", kvq.KV_INT4_BDR, 128, False, 2),
+               ("bdr128_kv_int2", kvq.KV_INT4_BDR, 128, True, 2)]
+    for name, mode, b, rv, bits in [v + (4,) for v in VARIANTS] + two_bit:
+        cache = kvq.PagedKVCache(w.num_pages, w.ps, w.H, w.Hq, mode, b, rv, device=device, fill=0, code_bits=bits)
         cache.append(k, v, ts, tp, w.page_table)
         out = cache.decode(w.q, w.seq_lens, w.dec_pt, w.max_len, out_fp32=True)
         status = cache.get_error()
@@ -499,6 +502,11 @@ def main():
                                   "decode_gbs": w.decode_bytes(kvq.KV_INT4_BDR) / (r["decode_ms"] / 1e3) / 1e9,
                                   "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3,
                                   "note": "plus the table reads (512 B per appended token, L2-resident)"}
+        # the 2-bit variant (half the code bytes: 576 B per token-layer instead of 1088)
+        r = run_variant(w, kvq.KV_INT4_BDR, 128, False, n, 3, device, code_bits=2)
+        sweep["bdr128_k_int2"] = {"append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
+                                  "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3,
+                                  "note": "2-bit codes; timed like the others, bytes not comparable"}
 
     accuracy = None
     if not args.no_accuracy and args.workload in ("batch16", "single256"):

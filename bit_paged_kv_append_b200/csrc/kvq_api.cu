@@ -55,6 +55,9 @@ kv_status kv_create_paged(const kv_desc* d, kv_cache** out) {
     if (d->mode != KV_BF16 && (!d->k_sz || !d->v_sz || !aligned(d->k_sz, 16) || !aligned(d->v_sz, 16)))
         return KV_ERR_INVALID;
     if (d->rope && (d->rope_positions < 1 || !aligned(d->rope, 16))) return KV_ERR_INVALID;
+    const int code_bits = d->code_bits == 0 ? 4 : d->code_bits;
+    if (code_bits != 4 && code_bits != 2) return KV_ERR_UNSUPPORTED;
+    if (code_bits == 2 && d->mode == KV_BF16) return KV_ERR_INVALID;
     const int64_t rows = int64_t(d->num_pages) * d->num_kv_heads * d->page_size;
     if (rows >= (int64_t(1) << 32)) return KV_ERR_INVALID;  // slot indices are 32-bit in the kernels
 
@@ -74,6 +77,7 @@ kv_status kv_create_paged(const kv_desc* d, kv_cache** out) {
     c->g.v_sz = static_cast<uint32_t*>(d->mode == KV_BF16 ? nullptr : d->v_sz);
     c->g.rope = d->rope;
     c->g.rope_positions = d->rope ? d->rope_positions : 0;
+    c->g.code_bits = d->mode == KV_BF16 ? 4 : code_bits;
     if (cudaGetDevice(&c->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess ||
         cudaMalloc(&c->err_dev, sizeof(int)) != cudaSuccess) {

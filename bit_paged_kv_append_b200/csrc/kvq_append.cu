@@ -59,6 +59,13 @@ constexpr uint32_t magic_pack_offset() {
     return c;
 }
 constexpr uint32_t kMagicPackOffset = magic_pack_offset();
+// ... and the offset of sixteen 2-bit codes packed with shifts of 2
+constexpr uint32_t magic_pack_offset2() {
+    uint32_t c = 0;
+    for (int k = 0; k < 16; ++k) c += kMagicBits << (2 * k);
+    return c;
+}
+constexpr uint32_t kMagicPackOffset2 = magic_pack_offset2();
 
 struct Params {
     CacheGeom g;
@@ -79,6 +86,15 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t (&u)[8]) {
 #pragma unroll
     for (int k = 6; k >= 0; --k) acc = (acc << 4) + u[k];
     return acc - kMagicPackOffset;
+}
+
+// Sixteen 2-bit codes (magic-biased float bits, element k in u[k]) -> one word, element k
+// in bits 2k, 2k + 1.
+__device__ __forceinline__ uint32_t pack16(const uint32_t (&u)[16]) {
+    uint32_t acc = u[15];
+#pragma unroll
+    for (int k = 14; k >= 0; --k) acc = (acc << 2) + u[k];
+    return acc - kMagicPackOffset2;
 }
 
 // Loads this thread's row from the swizzled stage into R[i] = (x_i, x_{i+64}).
@@ -152,6 +168,29 @@ __device__ __forceinline__ void quantise_pack(const float2 (&R)[64], float zf, f
     }
 }
 
+// 2-bit codes of a row into 8 packed words (the row's 32 bytes): word m < 4 holds elements
+// 16 m .. 16 m + 15 (R[.].x), word 4 + m elements 64 + 16 m .. (R[.].y).
+template <bool CLAMP>
+__device__ __forceinline__ void quantise_pack2(const float2 (&R)[64], float zf, float inv, uint32_t (&w)[8]) {
+    const float2 nz = make_float2(-zf, -zf), ii = make_float2(inv, inv), mm = make_float2(kMagic, kMagic);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        uint32_t ulo[16], uhi[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            float2 u = __ffma2_rn(__fadd2_rn(R[16 * m + k], nz), ii, mm);
+            if (CLAMP) {
+                u.x = u.x > kMagic ? fminf(u.x, kMagic + 3.0f) : kMagic;
+                u.y = u.y > kMagic ? fminf(u.y, kMagic + 3.0f) : kMagic;
+            }
+            ulo[k] = __float_as_uint(u.x);
+            uhi[k] = __float_as_uint(u.y);
+        }
+        w[m] = pack16(ulo);
+        w[4 + m] = pack16(uhi);
+    }
+}
+
 // min / max that return NaN when any input is NaN
 __device__ __forceinline__ float min_nan(float a, float b) {
     float d;
@@ -174,10 +213,12 @@ __device__ __forceinline__ float max3_nan(float a, float b, float c) {
     return d;
 }
 
-// Token-wise asymmetric INT4 of one row: writes 64 bytes of codes and the
-// (scale, zero) word.  A NaN anywhere in the row makes its min and max NaN:
-// every code 0, scale = zero = fp16 quiet NaN.
+// Token-wise asymmetric quantisation of one row with CB-bit codes (4: 64 bytes, 2: 32
+// bytes) and the (scale, zero) word.  A NaN anywhere in the row makes its min and max
+// NaN: every code 0, scale = zero = fp16 quiet NaN.
+template <int CB>
 __device__ __forceinline__ void quantise_store(const float2 (&R)[64], uint8_t* codes_dst, uint32_t* sz_dst) {
+    constexpr float kLevels = CB == 4 ? 15.0f : 3.0f;
     float mn4[4], mx4[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -194,14 +235,14 @@ __device__ __forceinline__ void quantise_store(const float2 (&R)[64], uint8_t* c
     if (mn != mn) {
         const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         st_global_v8(codes_dst, z);
-        st_global_v8(codes_dst + 32, z);
+        if (CB == 4) st_global_v8(codes_dst + 32, z);
         *sz_dst = 0x7E007E00u;
         return;
     }
     mn = __fadd_rn(mn, 0.0f);  // -0 + +0 = +0: canonical signed zero
     mx = __fadd_rn(mx, 0.0f);
     const float range = __fsub_rn(mx, mn);
-    const float s32 = __fdiv_rn(range, 15.0f);
+    const float s32 = __fdiv_rn(range, kLevels);
     const __half sh = __float2half_rn(s32);
     const __half zh = __float2half_rn(mn);
     const float sf = __half2float(sh);
@@ -211,14 +252,23 @@ __device__ __forceinline__ void quantise_store(const float2 (&R)[64], uint8_t* c
     // element needs clamping (an infinite scale or zero fails the test).
     const float umin = __fmaf_rn(__fsub_rn(mn, zf), inv, kMagic);
     const float umax = __fmaf_rn(__fsub_rn(mx, zf), inv, kMagic);
-    const bool in_range = (umin >= kMagic) && (umax <= kMagic + 15.0f);
-    uint32_t wa[8], wb[8];
-    if (in_range)
-        quantise_pack<false>(R, zf, inv, wa, wb);
-    else
-        quantise_pack<true>(R, zf, inv, wa, wb);
-    st_global_v8(codes_dst, wa);
-    st_global_v8(codes_dst + 32, wb);
+    const bool in_range = (umin >= kMagic) && (umax <= kMagic + kLevels);
+    if (CB == 4) {
+        uint32_t wa[8], wb[8];
+        if (in_range)
+            quantise_pack<false>(R, zf, inv, wa, wb);
+        else
+            quantise_pack<true>(R, zf, inv, wa, wb);
+        st_global_v8(codes_dst, wa);
+        st_global_v8(codes_dst + 32, wb);
+    } else {
+        uint32_t w[8];
+        if (in_range)
+            quantise_pack2<false>(R, zf, inv, w);
+        else
+            quantise_pack2<true>(R, zf, inv, w);
+        st_global_v8(codes_dst, w);
+    }
     *sz_dst = uint32_t(__half_as_ushort(sh)) | (uint32_t(__half_as_ushort(zh)) << 16);
 }
 
@@ -269,14 +319,14 @@ __device__ __forceinline__ void copy_row_rope(const uint8_t* stage, int row, con
     }
 }
 
-template <bool ROT, int BLK>
+template <bool ROT, int BLK, int CB>
 __device__ __forceinline__ void process_row(const uint8_t* stage, int row, float r_b, const float* cs,
                                             uint8_t* cdst, uint32_t* sdst) {
     float2 R[64];
     load_row(stage, row, R);
     if (cs) rope_row(R, cs);
     if (ROT) rotate_row<BLK>(R, r_b);
-    quantise_store(R, cdst, sdst);
+    quantise_store<CB>(R, cdst, sdst);
 }
 
 // BF16 cache: copy the row unchanged.
@@ -296,7 +346,7 @@ __device__ __forceinline__ void copy_row(const uint8_t* stage, int row, uint8_t*
     }
 }
 
-template <int MODE, int BLK, bool ROTV, bool ROPE>
+template <int MODE, int BLK, bool ROTV, bool ROPE, int CB>
 __global__ void __launch_bounds__(kThreads, 1)
     append_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, Params p) {
     extern __shared__ uint8_t smem_raw[];
@@ -428,10 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else
                         copy_row(stage, tid, dst);
                 } else {
-                    uint8_t* cdst = static_cast<uint8_t*>(kv ? p.g.v_pool : p.g.k_pool) + row * 64;
+                    uint8_t* cdst = static_cast<uint8_t*>(kv ? p.g.v_pool : p.g.k_pool) + row * (16 * CB);
                     uint32_t* sdst = (kv ? p.g.v_sz : p.g.k_sz) + row;
-                    if (kv == 0) process_row<MODE == 2, BLK>(stage, tid, p.r_b, ROPE ? cs : nullptr, cdst, sdst);
-                    else process_row<MODE == 2 && ROTV, BLK>(stage, tid, p.r_b, nullptr, cdst, sdst);
+                    if (kv == 0)
+                        process_row<MODE == 2, BLK, CB>(stage, tid, p.r_b, ROPE ? cs : nullptr, cdst, sdst);
+                    else
+                        process_row<MODE == 2 && ROTV, BLK, CB>(stage, tid, p.r_b, nullptr, cdst, sdst);
                 }
             }
             __syncwarp();
@@ -466,9 +518,9 @@ bool make_row_map(CUtensorMap* map, const void* base, int64_t rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int BLK, bool ROTV, bool ROPE>
+template <int MODE, int BLK, bool ROTV, bool ROPE, int CB>
 cudaError_t launch_r(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
-    auto kern = append_kernel<MODE, BLK, ROTV, ROPE>;
+    auto kern = append_kernel<MODE, BLK, ROTV, ROPE, CB>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
@@ -478,10 +530,16 @@ cudaError_t launch_r(const CUtensorMap& km, const CUtensorMap& vm, const Params&
     return launch_overlapped(kern, dim3(grid), dim3(kThreads), kSmemBytes, s, km, vm, p);
 }
 
+template <int MODE, int BLK, bool ROTV, bool ROPE>
+cudaError_t launch_c(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
+    if (MODE != 0 && p.g.code_bits == 2) return launch_r<MODE, BLK, ROTV, ROPE, 2>(km, vm, p, grid, s);
+    return launch_r<MODE, BLK, ROTV, ROPE, 4>(km, vm, p, grid, s);
+}
+
 template <int MODE, int BLK, bool ROTV>
 cudaError_t launch_t(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
-    return p.g.rope ? launch_r<MODE, BLK, ROTV, true>(km, vm, p, grid, s)
-                    : launch_r<MODE, BLK, ROTV, false>(km, vm, p, grid, s);
+    return p.g.rope ? launch_c<MODE, BLK, ROTV, true>(km, vm, p, grid, s)
+                    : launch_c<MODE, BLK, ROTV, false>(km, vm, p, grid, s);
 }
 
 }  // namespace

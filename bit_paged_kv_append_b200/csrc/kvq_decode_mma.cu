@@ -43,6 +43,9 @@
 //     operand takes its 8 columns as 4 heads x {high, low part of p scale}, so
 //     the low part costs no extra mma; two shuffles move each score from the
 //     q.K layout to the B layout.
+//   * 2-bit codes (the pages leave 2-bit open): the stage holds 32-byte rows; each
+//     load site reads half as many bytes and spreads them into the 4-bit nibble
+//     layout in registers, so every fragment mapping above is shared.
 //   * Which dimension and which token each fragment slot stands for is a fixed
 //     permutation chosen so that every thread reads contiguous bytes and the
 //     shared-memory reads are conflict-free; the output mapping undoes it.
@@ -61,6 +64,16 @@ constexpr int kOffV = kCodeBytes;          // stage layout: K codes | V codes | 
 constexpr int kOffKs = 2 * kCodeBytes;
 constexpr int kOffVs = 2 * kCodeBytes + kChunk * 4;
 constexpr int kStageBytes = 2 * kCodeBytes + 2 * kChunk * 4;  // 2176
+// Stage layout for CB-bit codes: K codes | V codes | K sz | V sz (2-bit rows are 32 bytes;
+// the 4-bit layout above is Stage<4>).
+template <int CB>
+struct Stage {
+    static constexpr int kRowBytes = 16 * CB;
+    static constexpr int kCode = kChunk * kRowBytes;
+    static constexpr int kOffV = kCode;
+    static constexpr int kOffKs = 2 * kCode;
+    static constexpr int kOffVs = 2 * kCode + kChunk * 4;
+};
 constexpr float kTwo24 = 16777216.0f;  // a masked nibble c in an fp16 lane is the subnormal c * 2^-24
 constexpr float kTwo20 = 1048576.0f;   // ... and a masked high nibble is 16 c * 2^-24 = c * 2^-20
 constexpr int kQFix = 8355711;  // |q_int| bound: 65536 hi + 256 mid + lo with hi, mid, lo in [-128, 127]
@@ -145,6 +158,17 @@ __device__ __forceinline__ int sigma(int n) { return n ^ ((n >> 2) & 1); }
 // bank groups.
 __device__ __forceinline__ int vrow_off(int r, int b) { return kOffV + 64 * r + (b ^ ((r & 2) << 4)); }
 
+// 2-bit codes -> the 4-bit nibble layout: byte b of w (codes of dims 4b .. 4b + 3 in bits
+// 2k, 2k + 1) becomes bytes 2b, 2b + 1 (dims 4b, 4b + 1 | 4b + 2, 4b + 3 in the low / high
+// nibbles), so the 4-bit fragment mappings apply unchanged.
+__device__ __forceinline__ uint32_t spread2(uint32_t t) {  // two bytes in 16-bit lanes
+    t = (t | (t << 4)) & 0x0F0F0F0Fu;
+    return (t | (t << 2)) & 0x33333333u;
+}
+__device__ __forceinline__ uint2 expand2(uint32_t w) {
+    return make_uint2(spread2(prmt(w, 0u, 0x4140u)), spread2(prmt(w, 0u, 0x4342u)));
+}
+
 // q' in fixed point (23 bits: q_int = rint(q' kQFix / max|q'|)) as three balanced signed
 // bytes, q_int = 65536 hi + 256 mid + lo.  Fewer bits (16: two bytes) cost up to ~2e-3
 // of the output on keys with outlier channels; 23 bits cost ~5e-6.
@@ -170,7 +194,9 @@ struct CtaRing {
 
 // One warp's 16-token chunks of its split: pool rows (one page-table lookup per lane,
 // 32 chunks a window) and the copies of chunk iw into a ring stage.
+template <int CB>
 struct ChunkStream {
+    using L = Stage<CB>;
     CtaRing* r;
     const int32_t* pt;  // this sequence's page-table row
     int t0, t1, nw, warp, lane, h;
@@ -227,14 +253,19 @@ struct ChunkStream {
             const bool ok = row != kNoRow;
             if (ok) {
                 const uint32_t d = dst0 + uint32_t(slot) * kStageBytes;
-                const int vsw = 16 * ((lane >> 2) & 2);  // this lane's V unit moves by 32 bytes
-                const uint8_t* ks = kc + size_t(row) * 64;
-                const uint8_t* vs = vc + size_t(row) * 64;
-                cp_async16_s(d, ks, pol);
-                cp_async16_s(d + 512, ks + 512, pol);
-                cp_async16_s((d + kOffV) ^ vsw, vs, pol);
-                cp_async16_s(((d + kOffV) ^ vsw) + 512, vs + 512, pol);
-                if (lane < 8) cp_async16_s(d + kOffKs, sz + row, pol);  // V words follow the K words
+                const uint8_t* ks = kc + size_t(row) * L::kRowBytes;
+                const uint8_t* vs = vc + size_t(row) * L::kRowBytes;
+                if (CB == 4) {
+                    const int vsw = 16 * ((lane >> 2) & 2);  // this lane's V unit moves by 32 bytes
+                    cp_async16_s(d, ks, pol);
+                    cp_async16_s(d + 512, ks + 512, pol);
+                    cp_async16_s((d + kOffV) ^ vsw, vs, pol);
+                    cp_async16_s(((d + kOffV) ^ vsw) + 512, vs + 512, pol);
+                } else {  // 512 bytes each: one copy per lane
+                    cp_async16_s(d, ks, pol);
+                    cp_async16_s(d + L::kOffV, vs, pol);
+                }
+                if (lane < 8) cp_async16_s(d + L::kOffKs, sz + row, pol);  // V words follow the K words
             }
             r->mask[warp][slot] = ok ? 0xFFFFu : 0u;  // the same value from every lane
         } else {
@@ -252,15 +283,21 @@ struct ChunkStream {
                 ok = page >= 0 && page < p.g.num_pages;
                 if (ok) {
                     const int64_t row = (int64_t(page) * p.g.H + h) * p.g.page_size + slot_of_pos(p, t);
-                    const int off = i * 64 + 32 * hf;
-                    const int voff = i * 64 + 32 * (hf ^ ((i >> 1) & 1));  // V rows swizzled (vrow_off)
-                    const uint8_t* kcp = kpool + row * 64 + 32 * hf;
-                    const uint8_t* vcp = vpool + row * 64 + 32 * hf;
-                    cp_async16(st + off, kcp, pol);
-                    cp_async16(st + off + 16, kcp + 16, pol);
-                    cp_async16(st + kOffV + voff, vcp, pol);
-                    cp_async16(st + kOffV + voff + 16, vcp + 16, pol);
-                    cp_async4(st + (hf ? kOffVs : kOffKs) + 4 * i, (hf ? p.g.v_sz : p.g.k_sz) + row);
+                    if (CB == 4) {
+                        const int off = i * 64 + 32 * hf;
+                        const int voff = i * 64 + 32 * (hf ^ ((i >> 1) & 1));  // V rows swizzled (vrow_off)
+                        const uint8_t* kcp = kpool + row * 64 + 32 * hf;
+                        const uint8_t* vcp = vpool + row * 64 + 32 * hf;
+                        cp_async16(st + off, kcp, pol);
+                        cp_async16(st + off + 16, kcp + 16, pol);
+                        cp_async16(st + kOffV + voff, vcp, pol);
+                        cp_async16(st + kOffV + voff + 16, vcp + 16, pol);
+                    } else {  // 32-byte rows: 16 bytes per lane of each
+                        const int off = i * 32 + 16 * hf;
+                        cp_async16(st + off, kpool + row * 32 + 16 * hf, pol);
+                        cp_async16(st + L::kOffV + off, vpool + row * 32 + 16 * hf, pol);
+                    }
+                    cp_async4(st + (hf ? L::kOffVs : L::kOffKs) + 4 * i, (hf ? p.g.v_sz : p.g.k_sz) + row);
                 } else if (hf == 0) {
                     flag_error(p.err, kErrOOB);
                 }
@@ -325,8 +362,9 @@ __device__ __forceinline__ void load_q_rotated(const DecodeParams& p, int s, int
 // Chunk's (scale, zero) words into floats, one word per lane (0..15 K, 16..31 V).
 // Values use centred codes c - 8, so their offset is zero + 8 scale; kscale
 // multiplies the key scales (exactly: a power of two).
+template <int CB>
 __device__ __forceinline__ void stage_szf(CtaRing& R, const uint8_t* st, int warp, int lane, float kscale) {
-    const uint32_t w = reinterpret_cast<const uint32_t*>(st + kOffKs)[lane];
+    const uint32_t w = reinterpret_cast<const uint32_t*>(st + Stage<CB>::kOffKs)[lane];
     const float sc = half_lo(w), zr = half_hi(w);
     R.szf[warp][lane >> 4][lane & 15] = lane < 16 ? make_float2(sc * kscale, zr) : make_float2(sc, zr + 8.0f * sc);
     __syncwarp();
@@ -336,13 +374,22 @@ __device__ __forceinline__ void stage_szf(CtaRing& R, const uint8_t* st, int war
 // (8 + tokA, 8 + tokB), bytes [8 gq, 8 gq + 8) of each row; row gq of tile jv is
 // dim 16 gq + 2 jv (low nibble), row gq + 8 is dim 16 gq + 2 jv + 1 (high nibble,
 // x16).  With kLow, (b0l, b1l) is accumulated by a second mma with the same A.
-template <bool kLow>
+template <bool kLow, int CB>
 __device__ __forceinline__ void pv_chunk(float (&O)[8][4], const uint8_t* st, int gq, int tokA, int tokB, uint32_t b0,
                                          uint32_t b1, uint32_t b0l, uint32_t b1l) {
-    const uint2 v00 = *reinterpret_cast<const uint2*>(st + vrow_off(tokA, 8 * gq));
-    const uint2 v01 = *reinterpret_cast<const uint2*>(st + vrow_off(tokB, 8 * gq));
-    const uint2 v10 = *reinterpret_cast<const uint2*>(st + vrow_off(8 + tokA, 8 * gq));
-    const uint2 v11 = *reinterpret_cast<const uint2*>(st + vrow_off(8 + tokB, 8 * gq));
+    uint2 v00, v01, v10, v11;
+    if (CB == 4) {
+        v00 = *reinterpret_cast<const uint2*>(st + vrow_off(tokA, 8 * gq));
+        v01 = *reinterpret_cast<const uint2*>(st + vrow_off(tokB, 8 * gq));
+        v10 = *reinterpret_cast<const uint2*>(st + vrow_off(8 + tokA, 8 * gq));
+        v11 = *reinterpret_cast<const uint2*>(st + vrow_off(8 + tokB, 8 * gq));
+    } else {  // dims 16 gq .. 16 gq + 15: 4 bytes of a 32-byte row, spread to the 4-bit layout
+        const uint8_t* vb = st + Stage<2>::kOffV + 4 * gq;
+        v00 = expand2(*reinterpret_cast<const uint32_t*>(vb + 32 * tokA));
+        v01 = expand2(*reinterpret_cast<const uint32_t*>(vb + 32 * tokB));
+        v10 = expand2(*reinterpret_cast<const uint32_t*>(vb + 32 * (8 + tokA)));
+        v11 = expand2(*reinterpret_cast<const uint32_t*>(vb + 32 * (8 + tokB)));
+    }
 #pragma unroll
     for (int wq = 0; wq < 2; ++wq) {
         const uint32_t x00 = wq ? v00.y : v00.x, x01 = wq ? v01.y : v01.x;
@@ -364,6 +411,15 @@ __device__ __forceinline__ void pv_chunk(float (&O)[8][4], const uint8_t* st, in
             }
         }
     }
+}
+
+// Codes of dims 32 pq .. 32 pq + 31 of token row tok in the 4-bit nibble layout (16 bytes).
+template <int CB>
+__device__ __forceinline__ uint4 key_codes(const uint8_t* st, int tok, int pq) {
+    if (CB == 4) return *reinterpret_cast<const uint4*>(st + tok * 64 + 16 * pq);
+    const uint2 r = *reinterpret_cast<const uint2*>(st + tok * 32 + 8 * pq);
+    const uint2 a = expand2(r.x), b = expand2(r.y);
+    return make_uint4(a.x, a.y, b.x, b.y);
 }
 
 // Merge scratch mo [warp][G][128]: each 16-byte chunk of a head's row is stored at chunk
@@ -409,7 +465,8 @@ __device__ __forceinline__ void store_partials(const DecodeParams& p, const floa
 }
 
 // Common start of a CTA: split bounds and the chunk stream.  False: no tokens.
-__device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, ChunkStream& cs, int warp, int lane,
+template <int CB>
+__device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, ChunkStream<CB>& cs, int warp, int lane,
                                             int tid) {
     const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int L = decode_len(p, s);
@@ -438,7 +495,7 @@ __device__ __forceinline__ bool begin_split(const DecodeParams& p, CtaRing& R, C
 // =====================================================================================
 // G = 8: heads on M, fp16 q.K
 // =====================================================================================
-template <int G>
+template <int G, int CB>
 __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p) {
     __shared__ __align__(128) CtaRing R;
     // q.K A operands (4 x s8 per word) in fragment order: m-tile 0 (rows hi | mid), [k-step][reg][lane];
@@ -449,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
     const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, pq = lane & 3;  // mma group id / thread in group
-    ChunkStream cs;
+    ChunkStream<CB> cs;
     if (!begin_split(p, R, cs, warp, lane, tid)) return;
     for (int w = tid; w < 4 * 4 * 32 + 4 * 2 * 32; w += kThreads) As[w] = 0u;
     __syncthreads();
@@ -527,13 +584,13 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         const uint8_t* st = R.stage[warp][slot];
         const uint32_t vmask = R.mask[warp][slot];
         const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
-        stage_szf(R, st, warp, lane, 1.0f);
+        stage_szf<CB>(R, st, warp, lane, 1.0f);
 
         // ---- scores: q_int . codes for the two 8-token n-tiles (column gq: token 8 tau + tokK) ----
         float C[2][2];
 #pragma unroll
         for (int tau = 0; tau < 2; ++tau) {
-            const uint4 kw = *reinterpret_cast<const uint4*>(st + (8 * tau + tokK) * 64 + 16 * pq);
+            const uint4 kw = key_codes<CB>(st, 8 * tau + tokK, pq);
             const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
             int D[4] = {0, 0, 0, 0}, E[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -607,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         const uint32_t b1 = pack_half2(pt_[1][0], pt_[1][1]);
         const uint32_t b0l = pack_half2(pt_[0][0] - half_lo(b0), pt_[0][1] - half_hi(b0));
         const uint32_t b1l = pack_half2(pt_[1][0] - half_lo(b1), pt_[1][1] - half_hi(b1));
-        pv_chunk<true>(O, st, gq, tokA, tokB, b0, b1, b0l, b1l);
+        pv_chunk<true, CB>(O, st, gq, tokA, tokB, b0, b1, b0l, b1l);
         __syncwarp();  // every lane is done with this slot
         if (i + kStages < nw) cs.issue(p, i + kStages, slot);
         cp_async_commit();
@@ -653,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
 // =====================================================================================
 // G <= 4: tokens on M, int8 q.K
 // =====================================================================================
-template <int G>
+template <int G, int CB>
 __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p) {
     static_assert(G >= 1 && G <= 4, "tokens-on-M tile serves up to 4 query heads per KV head");
     __shared__ __align__(128) CtaRing R;
@@ -665,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
     const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, pq = lane & 3;
-    ChunkStream cs;
+    ChunkStream<CB> cs;
     if (!begin_split(p, R, cs, warp, lane, tid)) return;
     for (int w = tid; w < 2 * 4 * 2 * 32; w += kThreads) Bs[w] = 0u;
     __syncthreads();
@@ -751,11 +808,11 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         const uint8_t* st = R.stage[warp][slot];
         const uint32_t vmask = R.mask[warp][slot];
         const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
-        stage_szf(R, st, warp, lane, 1.0f);
+        stage_szf<CB>(R, st, warp, lane, 1.0f);
 
         // ---- scores: codes (tokens tk, tk + 8; bytes [16 pq, 16 pq + 16)) . q_int ----
-        const uint4 k0 = *reinterpret_cast<const uint4*>(st + tk * 64 + 16 * pq);
-        const uint4 k1 = *reinterpret_cast<const uint4*>(st + (tk + 8) * 64 + 16 * pq);
+        const uint4 k0 = key_codes<CB>(st, tk, pq);
+        const uint4 k1 = key_codes<CB>(st, tk + 8, pq);
         const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
         int D[4] = {0, 0, 0, 0}, E[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -816,7 +873,7 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         // ---- to the P.V B layout: (tokA, tokB) and (tokA + 8, tokB + 8) of column gq ----
         const uint32_t R1 = __shfl_sync(kFull, part ? LO : HI, src1);
         const uint32_t R2 = __shfl_sync(kFull, part ? HI : LO, src2);
-        pv_chunk<false>(O, st, gq, tokA, tokB, prmt(R1, R2, sel0), prmt(R1, R2, sel1), 0u, 0u);
+        pv_chunk<false, CB>(O, st, gq, tokA, tokB, prmt(R1, R2, sel0), prmt(R1, R2, sel1), 0u, 0u);
         __syncwarp();  // every lane is done with this slot
         if (i + kStages < nw) cs.issue(p, i + kStages, slot);
         cp_async_commit();
@@ -853,11 +910,16 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
 
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s) {
     const dim3 grid(p.max_splits, p.g.H, p.a.batch);
+    const bool two = p.g.code_bits == 2;
     switch (p.g.Hq / p.g.H) {
-        case 1: return launch_overlapped(decode_tok_kernel<1>, grid, dim3(kThreads), 0, s, p);
-        case 2: return launch_overlapped(decode_tok_kernel<2>, grid, dim3(kThreads), 0, s, p);
-        case 4: return launch_overlapped(decode_tok_kernel<4>, grid, dim3(kThreads), 0, s, p);
-        case 8: return launch_overlapped(decode_mma_kernel<8>, grid, dim3(kThreads), 0, s, p);
+        case 1: return two ? launch_overlapped(decode_tok_kernel<1, 2>, grid, dim3(kThreads), 0, s, p)
+                           : launch_overlapped(decode_tok_kernel<1, 4>, grid, dim3(kThreads), 0, s, p);
+        case 2: return two ? launch_overlapped(decode_tok_kernel<2, 2>, grid, dim3(kThreads), 0, s, p)
+                           : launch_overlapped(decode_tok_kernel<2, 4>, grid, dim3(kThreads), 0, s, p);
+        case 4: return two ? launch_overlapped(decode_tok_kernel<4, 2>, grid, dim3(kThreads), 0, s, p)
+                           : launch_overlapped(decode_tok_kernel<4, 4>, grid, dim3(kThreads), 0, s, p);
+        case 8: return two ? launch_overlapped(decode_mma_kernel<8, 2>, grid, dim3(kThreads), 0, s, p)
+                           : launch_overlapped(decode_mma_kernel<8, 4>, grid, dim3(kThreads), 0, s, p);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -17,6 +17,7 @@ struct CacheGeom {
     uint32_t* v_sz;
     const float* rope;   // (cos, sin) [rope_positions][D/2][2], or nullptr
     int rope_positions;
+    int code_bits;       // INT4 modes: 4 or 2 (codes per byte: 8 / code_bits)
 };
 
 struct AppendArgs {

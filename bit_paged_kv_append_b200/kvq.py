@@ -36,7 +36,7 @@ class kv_desc(ctypes.Structure):
                 ("num_q_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("mode", ctypes.c_int),
                 ("bdr_block", ctypes.c_int), ("rotate_v", ctypes.c_int), ("k_pool", ctypes.c_void_p),
                 ("v_pool", ctypes.c_void_p), ("k_sz", ctypes.c_void_p), ("v_sz", ctypes.c_void_p),
-                ("rope", ctypes.c_void_p), ("rope_positions", ctypes.c_int)]
+                ("rope", ctypes.c_void_p), ("rope_positions", ctypes.c_int), ("code_bits", ctypes.c_int)]
 
 
 _lib = None
@@ -100,12 +100,13 @@ def _check(status: int, what: str):
 
 
 def kv_create_paged(num_pages, page_size, num_kv_heads, num_q_heads, head_dim, mode, bdr_block, rotate_v,
-                    k_pool, v_pool, k_sz=None, v_sz=None, rope=None) -> int:
+                    k_pool, v_pool, k_sz=None, v_sz=None, rope=None, code_bits=4) -> int:
     """Returns the opaque handle (an integer address); release it with kv_free.  rope: optional
-    device float32 [positions, head_dim/2, 2] (cos, sin) table (fused rotary embedding)."""
+    device float32 [positions, head_dim/2, 2] (cos, sin) table (fused rotary embedding);
+    code_bits: 4 or 2 for the INT4 modes."""
     d = kv_desc(num_pages, page_size, num_kv_heads, num_q_heads, head_dim, mode, bdr_block, int(bool(rotate_v)),
                 _ptr(k_pool), _ptr(v_pool), _ptr(k_sz), _ptr(v_sz), _ptr(rope),
-                int(rope.shape[0]) if rope is not None else 0)
+                int(rope.shape[0]) if rope is not None else 0, int(code_bits))
     h = ctypes.c_void_p()
     _check(load().kv_create_paged(ctypes.byref(d), ctypes.byref(h)), "kv_create_paged")
     return h.value
@@ -152,7 +153,7 @@ def kv_free(cache):
 
 # ---- device-memory plumbing (torch allocations in the documented layouts) ----
 
-def alloc_pools(num_pages, page_size, num_kv_heads, mode, device="cuda", fill: int | None = None):
+def alloc_pools(num_pages, page_size, num_kv_heads, mode, device="cuda", fill: int | None = None, code_bits=4):
     """Caller-owned pools for a cache: (k_pool, v_pool, k_sz, v_sz); sz is None in BF16 mode."""
     if mode == KV_BF16:
         shape = (num_pages, num_kv_heads, page_size, HEAD_DIM)
@@ -160,7 +161,7 @@ def alloc_pools(num_pages, page_size, num_kv_heads, mode, device="cuda", fill: i
         v = torch.empty(shape, dtype=torch.bfloat16, device=device)
         ks = vs = None
     else:
-        shape = (num_pages, num_kv_heads, page_size, HEAD_DIM // 2)
+        shape = (num_pages, num_kv_heads, page_size, HEAD_DIM * code_bits // 8)
         k = torch.empty(shape, dtype=torch.uint8, device=device)
         v = torch.empty(shape, dtype=torch.uint8, device=device)
         ks = torch.empty((num_pages, num_kv_heads, page_size, 2), dtype=torch.float16, device=device)
@@ -176,15 +177,16 @@ class PagedKVCache:
     """Owns one handle over caller-provided (or freshly allocated) pools."""
 
     def __init__(self, num_pages, page_size, num_kv_heads, num_q_heads, mode, bdr_block=128, rotate_v=False,
-                 pools=None, device="cuda", fill=None, rope=None):
+                 pools=None, device="cuda", fill=None, rope=None, code_bits=4):
         self.mode, self.bdr_block, self.rotate_v = mode, bdr_block, bool(rotate_v)
         self.rope = rope  # kept alive with the handle
+        self.code_bits = code_bits
         self.num_pages, self.page_size = num_pages, page_size
         self.num_kv_heads, self.num_q_heads = num_kv_heads, num_q_heads
         self.k_pool, self.v_pool, self.k_sz, self.v_sz = pools or alloc_pools(num_pages, page_size, num_kv_heads,
-                                                                               mode, device, fill)
+                                                                               mode, device, fill, code_bits)
         self.handle = kv_create_paged(num_pages, page_size, num_kv_heads, num_q_heads, HEAD_DIM, mode, bdr_block,
-                                      rotate_v, self.k_pool, self.v_pool, self.k_sz, self.v_sz, rope)
+                                      rotate_v, self.k_pool, self.v_pool, self.k_sz, self.v_sz, rope, code_bits)
 
     def append(self, k, v, tok_seq, tok_pos, page_table, stream=None):
         kv_append_quant(self.handle, k, v, k.shape[0], tok_seq, tok_pos, page_table, page_table.shape[1],

@@ -37,6 +37,7 @@
  *
  * Memory layout (all buffers are caller-owned device memory):
  *  INT4 pools   uint8  [num_pages, num_kv_heads, page_size, head_dim/2]
+ *               (head_dim/4 with code_bits = 2: four 2-bit codes per byte)
  *  scale/zero   fp16x2 [num_pages, num_kv_heads, page_size] (scale, zero)
  *  BF16 pools   bf16   [num_pages, num_kv_heads, page_size, head_dim]
  *  page_table   int32  [num_seqs, pt_stride]; token p of sequence s lives in
@@ -102,6 +103,10 @@ typedef struct {
      * zero output), flagged KV_ERR_OOB. */
     const float* rope;
     int rope_positions; /* rows of the table (>= 1 when rope is set) */
+    /* Code width of the INT4 modes: 0 or 4 = 4-bit codes; 2 = the 2-bit variant (the
+     * same token-wise asymmetric quantiser with range/3, codes 0..3, four per byte,
+     * code k of a byte in bits 2k and 2k+1; the pages leave 2-bit open). */
+    int code_bits;
 } kv_desc;
 
 typedef struct kv_cache kv_cache; /* opaque host handle */

@@ -51,10 +51,11 @@ class Case:
     cache: kvq.PagedKVCache = None
     ref_pools: tuple = None
     rope: torch.Tensor = None  # optional (cos, sin) table, float32 [positions, 64, 2] on the CPU
+    code_bits: int = 4
 
 
 def make_case(mode, bdr, rotate_v, lengths, wl: synth.Workload, seed=0, spare_pages=3, device="cuda",
-              starts=None, capacities=None, rope=None):
+              starts=None, capacities=None, rope=None, code_bits=4):
     T = sum(lengths)
     k, v = synth.make_kv(T, wl, seed)
     caps = capacities or [st + n for st, n in zip(starts or [0] * len(lengths), lengths)]
@@ -62,8 +63,10 @@ def make_case(mode, bdr, rotate_v, lengths, wl: synth.Workload, seed=0, spare_pa
     ts, tp = synth.append_positions(lengths, starts)
     c = Case(mode, bdr, rotate_v, wl, lengths, k, v, ts, tp, pt, P)
     c.rope = rope
+    c.code_bits = code_bits
     c.cache = kvq.PagedKVCache(P, wl.page_size, wl.num_kv_heads, wl.num_q_heads, mode, bdr, rotate_v,
-                               device=device, fill=FILL, rope=None if rope is None else rope.to(device))
+                               device=device, fill=FILL, rope=None if rope is None else rope.to(device),
+                               code_bits=code_bits)
     return c
 
 
@@ -83,7 +86,7 @@ def oracle_pools(c: Case):
         vp = kp.copy()
         ks = vs = np.zeros(1, dtype=np.uint16)
     else:
-        kp = np.full((P, H, ps, 64), FILL, dtype=np.uint8)
+        kp = np.full((P, H, ps, 16 * c.code_bits), FILL, dtype=np.uint8)
         vp = kp.copy()
         ks = np.full((P, H, ps, 2), FILL * 257, dtype=np.uint16)
         vs = ks.copy()
@@ -96,7 +99,7 @@ def oracle_append(c: Case, pools=None, k=None, v=None, ts=None, tp=None):
     skipped = oracle.append(c.mode, c.bdr, c.rotate_v, kp, vp, ks, vs, bits16(c.k if k is None else k),
                             bits16(c.v if v is None else v), (c.tok_seq if ts is None else ts).numpy(),
                             (c.tok_pos if tp is None else tp).numpy(), c.page_table.numpy(),
-                            rope=None if c.rope is None else c.rope.numpy())
+                            rope=None if c.rope is None else c.rope.numpy(), code_bits=c.code_bits)
     c.ref_pools = pools
     return skipped
 
@@ -132,7 +135,8 @@ def oracle_decode(c: Case, q, seq_lens, rows=None, page_table=None):
     kp, vp, ks, vs = c.ref_pools
     pt = (c.page_table if page_table is None else page_table).numpy()
     return oracle.decode(c.mode, c.bdr, c.rotate_v, kp, vp, ks, vs, bits16(q), np.asarray(seq_lens), pt,
-                         c.wl.num_kv_heads, rows=rows, rope=None if c.rope is None else c.rope.numpy())
+                         c.wl.num_kv_heads, rows=rows, rope=None if c.rope is None else c.rope.numpy(),
+                         code_bits=c.code_bits)
 
 
 def attn_rel_err(got: np.ndarray, ref: np.ndarray) -> float:

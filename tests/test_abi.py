@@ -65,6 +65,8 @@ def _desc(**kw):
     (dict(k_sz=0), kvq.KV_ERR_INVALID),
     (dict(rope=0x5000, rope_positions=0), kvq.KV_ERR_INVALID),  # a table needs >= 1 row
     (dict(rope=0x5004, rope_positions=8), kvq.KV_ERR_INVALID),  # not 16-byte aligned
+    (dict(code_bits=3), kvq.KV_ERR_UNSUPPORTED),
+    (dict(code_bits=2, mode=kvq.KV_BF16), kvq.KV_ERR_INVALID),
 ])
 def test_create_rejects_bad_descriptors(kw, status):
     lib = kvq.load()
