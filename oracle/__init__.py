@@ -14,7 +14,8 @@ fused into paged KV-cache layouts) and the wispaper.ai blog's sections 2-3
 query rotated in step at decode).
 
 Parity status: every exported function is pinned by ``tests/test_oracle_pins.py``
-against closed forms, invariants, special cases or brute force on tiny inputs.
+(and ``extend`` by ``tests/test_oracle_extend.py``) against closed forms,
+invariants, special cases or brute force on tiny inputs.
 """
 from __future__ import annotations
 
@@ -201,3 +202,35 @@ def decode(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz
     if rows is None:
         out = out.reshape(B, Hq, D)
     return out, int(skipped)
+
+
+def extend_lengths(q_indptr, seq_lens) -> tuple[np.ndarray, np.ndarray]:
+    """Per query row of an extend call: (its sequence, its decode length = position + 1).
+
+    Query i (0-based) of the n_s = q_indptr[s+1] - q_indptr[s] newest tokens of sequence s
+    sits at position seq_lens[s] - n_s + i: the new tokens are the last n_s of the
+    sequence, in order."""
+    qi = np.asarray(q_indptr, dtype=np.int64)
+    n = np.diff(qi)
+    seq_of = np.repeat(np.arange(len(n)), n)
+    i_in = np.arange(int(qi[-1])) - qi[seq_of]
+    lens = np.asarray(seq_lens, dtype=np.int64)[seq_of] - n[seq_of] + i_in + 1
+    return seq_of, lens
+
+
+def extend(mode: int, bdr_block: int, rotate_v: bool, k_pool, v_pool, k_sz, v_sz, q_bits, q_indptr, seq_lens,
+           page_table, num_kv_heads: int, rows=None, rope=None, code_bits: int = 4):
+    """Extend (chunked-prefill) attention in float64: causal attention of each sequence's
+    newest tokens over the paged cache (the SAW-INT4 abstract: attention executed over the
+    paged quantised cache; the wispaper.ai blog, section 3: the query rotated in step).
+
+    The query at position p attends to tokens 0 .. p, which is the decode attention of a
+    sequence of length p + 1 (query turned by the rotary table at p): this function is that
+    definition, one decode row per (query, head).  q_bits: bf16 bits uint16 [total_q, Hq, D];
+    rows: optional [(query row, query head), ...].  Returns (out float64 [n, D] or
+    [total_q, Hq, D], skipped-token count)."""
+    seq_of, lens = extend_lengths(q_indptr, seq_lens)
+    lens = np.clip(lens, -1, np.iinfo(np.int32).max).astype(np.int32)  # <= 0: no tokens (zero row)
+    pt = np.ascontiguousarray(np.asarray(page_table, dtype=np.int32)[seq_of])
+    return decode(mode, bdr_block, rotate_v, k_pool, v_pool, k_sz, v_sz, q_bits, lens, pt, num_kv_heads,
+                  rows=rows, rope=rope, code_bits=code_bits)
