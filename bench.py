@@ -44,6 +44,7 @@ from bit_paged_kv_append_b200 import kvq, synth  # noqa: E402
 METRIC = "INT4+BDR KV append tokens/s; paged decode attn HBM GB/s (% of ~8 TB/s)"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 VARIANTS = [("bf16", kvq.KV_BF16, 0, False), ("int4", kvq.KV_INT4, 0, False)] + [
     (f"bdr{b}_{'kv' if rv else 'k'}", kvq.KV_INT4_BDR, b, rv) for b in (16, 32, 64, 128) for rv in (False, True)]
@@ -53,9 +54,20 @@ HEADLINE = {"batch16": ("bdr128_k", kvq.KV_INT4_BDR, 128, False),
             "decode64x8k": ("bdr128_k", kvq.KV_INT4_BDR, 128, False),
             "mixed256": ("bdr128_kv", kvq.KV_INT4_BDR, 128, True),
             "long1m": ("bdr128_k", kvq.KV_INT4_BDR, 128, False)}
-_DECODE_SOURCES = ["kvq_decode_mma.cu", "kvq_decode.cuh", "kvq_common.cuh", "kvq_internal.h"]
+_DECODE_SOURCES = ["kvq_decode_mma.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh", "kvq_internal.h"]
 KERNEL_SOURCES = {"append_kernel": ["kvq_append.cu", "kvq_common.cuh", "kvq_internal.h"],
-                  "decode_tok_kernel": _DECODE_SOURCES, "decode_mma_kernel": _DECODE_SOURCES}
+                  "decode_tok_kernel": _DECODE_SOURCES, "decode_mma_kernel": _DECODE_SOURCES,
+                  "extend_kernel": ["kvq_extend.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh",
+                                    "kvq_internal.h"]}
+
+
+def peak_bf16_tflops():
+    """Dense bf16 tensor peak, burst figure (a kernel timed alone)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def peak_hbm():
@@ -113,6 +125,7 @@ class Workload:
         elif name == "mixed256":
             rng = np.random.default_rng(seed + 7)
             prefilling = set(rng.choice(B, 8, replace=False).tolist())
+            self.prefilling = sorted(prefilling)
             self.prefill = [(lengths, [0] * B)]
             step = [([2048 if s in prefilling else 1 for s in range(B)], lengths)]
             dec_seqs = [s for s in range(B) if s not in prefilling]
@@ -280,6 +293,70 @@ def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False, r
             "append_ms_median": float(np.median(app)), "decode_ms_median": float(np.median(dec)),
             "wall_s": wall, "status": status, "clocks": sampler.summary() if sampler else None,
             "launches_per_step": len(w.appends) + 2}
+
+
+def extend_setup(w: Workload):
+    """The step's prefill attention: (sequences, their cached lengths after the step's append,
+    new queries per sequence).  mixed256: the 8 sequences that append a 2048-token chunk attend
+    over it; batch16 / single256: every sequence, appended from position 0, is one prefill."""
+    if w.name == "mixed256":
+        return w.prefilling, [w.lengths[s] + 2048 for s in w.prefilling], [2048] * len(w.prefilling)
+    if w.name in ("batch16", "single256"):
+        return list(range(len(w.lengths))), list(w.lengths), list(w.lengths)
+    return None
+
+
+def run_extend(w: Workload, mode, b, rv, reps, device):
+    """kv_extend_attn over the step's prefill queries (after the step's append), CUDA events around
+    each launch on the launching stream, L2 flushed between launches.  Work: 4 D flops per
+    (query head, attended token) -- the q.K and P.V of bf16 attention, to compare with the dense
+    bf16 tensor peak; bytes: each sequence's cached codes + scale/zero read once, q and out."""
+    seqs, lens, qlens = extend_setup(w)
+    cache = make_cache(w, mode, b, rv, device)
+    for k, v, ts, tp in w.appends:
+        cache.append(k, v, ts, tp, w.page_table)
+    nq = sum(qlens)
+    q = synth.make_q(nq, w.Hq, 128, w.seed + 99, device=device)
+    qi = torch.tensor(np.concatenate([[0], np.cumsum(qlens)]), dtype=torch.int32, device=device)
+    sl = torch.tensor(lens, dtype=torch.int32, device=device)
+    pt = w.page_table[torch.tensor(seqs, device=device)].contiguous()
+    out = torch.empty(nq, w.Hq, 128, dtype=torch.bfloat16, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def launch():
+        kvq.kv_extend_attn(cache.handle, q, qi, sl, pt, w.pt_stride, len(seqs), max(qlens), max(lens), out, 0, stream)
+
+    for _ in range(3):
+        flush.zero_()
+        launch()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        launch()
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = np.array([e0.elapsed_time(e1) for e0, e1 in evs])
+    status = cache.get_error()
+    cache.close()
+    attended = sum(n * (L - n) + n * (n + 1) // 2 for L, n in zip(lens, qlens))  # sum over queries of position + 1
+    flops = 4 * 128 * w.Hq * attended
+    per_tok = w.H * (2 * 68 if mode != kvq.KV_BF16 else 2 * 256)
+    nbytes = sum(lens) * per_tok + nq * w.Hq * 128 * 2 * 2
+    peak, kind = peak_bf16_tflops()
+    t = float(ms.mean())
+    return {"us": t * 1e3, "us_median": float(np.median(ms)) * 1e3, "launches": reps, "sequences": len(seqs),
+            "queries": nq, "query_heads": w.Hq, "attended_tokens_per_query_head": attended,
+            "flops": flops, "tflops": flops / (t / 1e3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "extend_kernel", "achieved": flops / (t / 1e3) / 1e12,
+                         "peak": peak, "unit": "TFLOP/s", "frac": flops / (t / 1e3) / 1e12 / peak,
+                         "peak_source": f"{kind} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops); the kernel "
+                                        "runs int8 (q.K) and fp16 (P.V) mma.sync tiles",
+                         "traffic": profiled_traffic("extend_kernel", w.name)},
+            "algorithmic_bytes": nbytes, "gbs": nbytes / (t / 1e3) / 1e9,
+            "device_status": kvq.status_string(status)}
 
 
 def exact_attention(k, v, q, lengths, H, Hq):
@@ -462,6 +539,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-accuracy", action="store_true")
+    ap.add_argument("--no-extend", action="store_true")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -507,6 +585,10 @@ def main():
         sweep["bdr128_k_int2"] = {"append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
                                   "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3,
                                   "note": "2-bit codes; timed like the others, bytes not comparable"}
+
+    extend = None
+    if not args.no_extend and extend_setup(w) is not None:
+        extend = run_extend(w, hmode, hb, hrv, 10, device)
 
     accuracy = None
     if not args.no_accuracy and args.workload in ("batch16", "single256"):
@@ -555,6 +637,9 @@ def main():
     }
     if sweep:
         line["sweep"] = sweep
+    if extend:
+        line["extend"] = {"what": "kv_extend_attn: causal attention of the step's prefill queries over the "
+                                  "paged cache (one launch), outside the timed step", **extend}
     if accuracy:
         line["accuracy"] = {"vs": "exact float64 attention on the unquantised bf16 K/V",
                             "metric": "per (sequence, query head) row max|o-r|/max|r|", **accuracy}

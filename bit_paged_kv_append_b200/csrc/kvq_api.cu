@@ -1,6 +1,6 @@
 // kvq_api.cu -- the C ABI of libkvq.so (declared in include/kvq.h): host-side
 // validation, the opaque handle, the device error word, and dispatch to the
-// append / decode launchers.  No kernel is launched before every argument has
+// append / decode / extend launchers.  No kernel is launched before every argument has
 // been checked; nothing here allocates on the per-call path.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -126,6 +126,24 @@ kv_status kv_decode_attn(kv_cache* c, const void* q, const int32_t* seq_lens, co
     kvq::DecodeArgs a{q, seq_lens, page_table, pt_stride, batch, max_seq_len, out, out_fp32 ? 1 : 0,
                       workspace, workspace_bytes};
     cudaError_t e = kvq::launch_decode(c->g, a, plan, c->err_dev, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+kv_status kv_extend_attn(kv_cache* c, const void* q, const int32_t* q_indptr, const int32_t* seq_lens,
+                         const int32_t* page_table, int pt_stride, int batch, int max_q_len, int max_seq_len,
+                         void* out, int out_fp32, void* stream) {
+    if (!c || batch < 0 || max_q_len < 0 || max_seq_len < 0) return KV_ERR_INVALID;
+    if (batch == 0 || max_q_len == 0) return KV_OK;
+    if (!q || !q_indptr || !seq_lens || !page_table || !out || pt_stride < 1) return KV_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(q_indptr, 4) || !aligned(seq_lens, 4) || !aligned(page_table, 4) ||
+        !aligned(out, 16))
+        return KV_ERR_INVALID;
+    if (c->g.mode == KV_BF16) return KV_ERR_UNSUPPORTED;
+    const int qb = kvq::extend_queries_per_cta(c->g);
+    if (batch > 65535 || (max_q_len + qb - 1) / qb > 65535) return KV_ERR_UNSUPPORTED;  // grid extents
+    kvq::ExtendArgs a{q, q_indptr, seq_lens, page_table, pt_stride, batch, max_q_len, max_seq_len, out,
+                      out_fp32 ? 1 : 0};
+    cudaError_t e = kvq::launch_extend(c->g, a, c->err_dev, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 

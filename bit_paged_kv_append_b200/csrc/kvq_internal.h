@@ -44,6 +44,19 @@ struct DecodeArgs {
     size_t workspace_bytes;
 };
 
+struct ExtendArgs {
+    const void* q;
+    const int32_t* q_indptr;  // [batch + 1]: queries of sequence s are rows q_indptr[s] .. q_indptr[s + 1] - 1
+    const int32_t* seq_lens;
+    const int32_t* page_table;
+    int pt_stride;
+    int batch;
+    int max_q_len;
+    int max_seq_len;
+    void* out;
+    int out_fp32;
+};
+
 // Split-K plan for one decode call: cached tokens per work item, the bound on
 // items per sequence and in total, and the workspace they need.
 struct DecodePlan {
@@ -60,5 +73,9 @@ DecodePlan plan_decode(const CacheGeom& g, int batch, int max_seq_len, int num_s
 cudaError_t launch_append(const CacheGeom& g, const AppendArgs& a, int* err_word, int num_sms, cudaStream_t s);
 cudaError_t launch_decode(const CacheGeom& g, const DecodeArgs& a, const DecodePlan& plan, int* err_word,
                           cudaStream_t s);
+// INT4 modes only (the caller rejects BF16 pages).
+cudaError_t launch_extend(const CacheGeom& g, const ExtendArgs& a, int* err_word, cudaStream_t s);
+// Query rows one extend CTA covers for this cache (grid extent along the queries: max_q_len / this).
+int extend_queries_per_cta(const CacheGeom& g);
 
 }  // namespace kvq

@@ -64,6 +64,8 @@ def load(path: str | None = None, build_if_missing: bool = True):
     lib.kv_decode_attn.restype = I
     lib.kv_decode_attn_noalloc.argtypes = [P, P, P, P, I, I, I, P, I, P]
     lib.kv_decode_attn_noalloc.restype = I
+    lib.kv_extend_attn.argtypes = [P, P, P, P, P, I, I, I, I, P, I, P]
+    lib.kv_extend_attn.restype = I
     lib.kv_get_error.argtypes = [P, P]
     lib.kv_get_error.restype = I
     lib.kv_free.argtypes = [P]
@@ -141,6 +143,13 @@ def kv_decode_attn_noalloc(cache, q, seq_lens, page_table, pt_stride, batch, max
                                          _stream(stream)), "kv_decode_attn_noalloc")
 
 
+def kv_extend_attn(cache, q, q_indptr, seq_lens, page_table, pt_stride, batch, max_q_len, max_seq_len, out,
+                   out_fp32, stream=None):
+    _check(load().kv_extend_attn(cache, _ptr(q), _ptr(q_indptr), _ptr(seq_lens), _ptr(page_table), int(pt_stride),
+                                 int(batch), int(max_q_len), int(max_seq_len), _ptr(out), int(bool(out_fp32)),
+                                 _stream(stream)), "kv_extend_attn")
+
+
 def kv_get_error(cache, stream=None) -> int:
     """Synchronises the stream; returns (does not raise) KV_OK, KV_ERR_OOB or KV_ERR_TIMEOUT."""
     return int(load().kv_get_error(cache, _stream(stream)))
@@ -206,6 +215,15 @@ class PagedKVCache:
         ws, n = workspace
         kv_decode_attn(self.handle, q, seq_lens, page_table, page_table.shape[1], B, max_seq_len, out, out_fp32,
                        ws, ws.numel(), stream)
+        return out
+
+    def extend(self, q, q_indptr, seq_lens, page_table, max_q_len, max_seq_len, out=None, out_fp32=False,
+               stream=None):
+        """Causal attention of each sequence's newest q_indptr[s+1] - q_indptr[s] tokens (rows of q)."""
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+        kv_extend_attn(self.handle, q, q_indptr, seq_lens, page_table, page_table.shape[1], seq_lens.shape[0],
+                       max_q_len, max_seq_len, out, out_fp32, stream)
         return out
 
     def get_error(self, stream=None) -> int:

@@ -182,6 +182,32 @@ kv_status kv_decode_attn_noalloc(kv_cache* cache, const void* q, const int32_t* 
                                  const int32_t* page_table, int pt_stride, int batch, int max_seq_len,
                                  void* out, int out_fp32, void* stream);
 
+/* Extend (chunked-prefill) attention over the INT4 cache: the n_s newest tokens of
+ * sequence s, already written by kv_append_quant, attend causally to the cached
+ * tokens ([ABS]: fused attention execution over the paged quantised cache, which
+ * chunked prefill in mixed serving reads this way).  Query i (0-based) of sequence s
+ * sits at position p = seq_lens[s] - n_s + i and its output row is exactly what
+ * kv_decode_attn gives for that query with seq_len = p + 1: q turned by the rotary
+ * table at position p (when set), rotated with H_blk ([WIS3]), softmax over tokens
+ * 0 .. p, output rotated back when values are rotated.
+ *  q           device bf16 [total_q, num_q_heads, head_dim], total_q = q_indptr[batch]
+ *  q_indptr    device int32 [batch + 1], non-decreasing, q_indptr[0] = 0: the queries
+ *              of sequence s are rows q_indptr[s] .. q_indptr[s + 1] - 1 of q and out
+ *  seq_lens    device int32 [batch]: cached tokens of s, its new ones included
+ *  page_table  device int32 [batch, pt_stride]
+ *  max_q_len   >= every n_s (host bound; sizes the grid), max_seq_len >= every seq_len
+ *  out         device [total_q, num_q_heads, head_dim], bf16 (round to nearest even of
+ *              the fp32 value) or fp32 (out_fp32 != 0)
+ * No workspace; one launch.  KV_BF16 pages: KV_ERR_UNSUPPORTED.  batch > 65535 or
+ * max_q_len above 65535 blocks of 64 / G queries: KV_ERR_UNSUPPORTED.  Flagged
+ * (KV_ERR_OOB via kv_get_error): n_s > max_q_len (the queries before the last
+ * max_q_len ones are not computed), p < 0 (n_s > seq_len: zero row), p outside the
+ * rotary table (zero row), p + 1 beyond the page table or max_seq_len (clamped as in
+ * kv_decode_attn), page ids outside the pool (token skipped). */
+kv_status kv_extend_attn(kv_cache* cache, const void* q, const int32_t* q_indptr, const int32_t* seq_lens,
+                         const int32_t* page_table, int pt_stride, int batch, int max_q_len, int max_seq_len,
+                         void* out, int out_fp32, void* stream);
+
 /* Synchronise the stream, then read and clear the device error word:
  * KV_OK, KV_ERR_OOB or KV_ERR_TIMEOUT (KV_ERR_CUDA if the runtime failed). */
 kv_status kv_get_error(kv_cache* cache, void* stream);

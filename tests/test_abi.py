@@ -81,6 +81,7 @@ def test_null_arguments_are_rejected():
     assert lib.kv_create_paged(None, None) == kvq.KV_ERR_INVALID
     assert lib.kv_append_quant(None, None, None, 1, None, None, None, 1, 1, None) == kvq.KV_ERR_INVALID
     assert lib.kv_decode_attn(None, None, None, None, 1, 1, 1, None, 0, None, 0, None) == kvq.KV_ERR_INVALID
+    assert lib.kv_extend_attn(None, None, None, None, None, 1, 1, 1, 1, None, 0, None) == kvq.KV_ERR_INVALID
     assert lib.kv_get_error(None, None) == kvq.KV_ERR_INVALID
     assert lib.kv_decode_workspace_bytes(None, 1, 1) == 0
     lib.kv_free(None)
