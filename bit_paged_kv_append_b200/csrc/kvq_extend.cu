@@ -30,6 +30,8 @@
 //     chunks the P.V accumulators are folded into a shared-memory copy with ordinary fp32
 //     arithmetic (scaled to the current row maxima) and restarted from zero, which bounds
 //     each accumulator's run as the decode's split length does.
+#include <type_traits>
+
 #include "kvq_mma.cuh"
 
 namespace kvq {
@@ -224,105 +226,121 @@ __global__ void __launch_bounds__(kThreads, 2) extend_kernel(ExtendParams ep) {
 
         // ---- q_int . codes: column gq of n-tile tau is token 8 tau + tokK ----
         int X[2][4], Y[2][4], W[2][4];
+        uint32_t kwv[2][4];
 #pragma unroll
         for (int tau = 0; tau < 2; ++tau) {
+            const uint4 kw = key_codes<CB>(st, 8 * tau + tokK, pq);
+            kwv[tau][0] = kw.x;
+            kwv[tau][1] = kw.y;
+            kwv[tau][2] = kw.z;
+            kwv[tau][3] = kw.w;
 #pragma unroll
             for (int c = 0; c < 4; ++c) X[tau][c] = Y[tau][c] = W[tau][c] = 0;
-            const uint4 kw = key_codes<CB>(st, 8 * tau + tokK, pq);
-            const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
+        }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t b0 = w[j] & 0x0F0F0F0Fu, b1 = (w[j] >> 4) & 0x0F0F0F0Fu;
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau) {  // six independent accumulators between dependent mmas
+                const uint32_t b0 = kwv[tau][j] & 0x0F0F0F0Fu, b1 = (kwv[tau][j] >> 4) & 0x0F0F0F0Fu;
                 mma16832_s8u8(X[tau], A[0][j], b0, b1);
                 mma16832_s8u8(Y[tau], A[1][j], b0, b1);
                 mma16832_s8u8(W[tau], A[2][j], b0, b1);
             }
-        }
-        // A chunk below every row's length and on valid pages needs no per-token masks.
-        const bool full = (tb + kChunk <= tmin) && (vmask == 0xFFFFu);
-        float sc[2][2][2];  // [row half][tau][column 2 pq + e]
-#pragma unroll
-        for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int lt = 8 * tau + (e ? tokB : tokA);
-                const float2 kz = R.szf[warp][0][lt];
-                const float c0 = q_dot(X[tau][e], X[tau][2 + e], W[tau][e]);
-                const float c1 = q_dot(Y[tau][e], Y[tau][2 + e], W[tau][2 + e]);
-                const bool page_ok = ((vmask >> lt) & 1u) != 0;
-                const bool ok0 = full || (page_ok && tb + lt < len[0]);
-                const bool ok1 = full || (page_ok && tb + lt < len[1]);
-                sc[0][tau][e] = ok0 ? qsc[0] * fmaf(kz.x, c0, kz.y * qsn[0]) : -INFINITY;
-                sc[1][tau][e] = ok1 ? qsc[1] * fmaf(kz.x, c1, kz.y * qsn[1]) : -INFINITY;
-            }
-        // ---- online softmax (log2 domain) per row; a row's 16 scores sit in one lane quad ----
-        float mn[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            float cm = fmaxf(fmaxf(sc[t][0][0], sc[t][0][1]), fmaxf(sc[t][1][0], sc[t][1][1]));
-            cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 1));
-            cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 2));
-            mn[t] = fmaxf(m[t], cm);
-        }
-        if (__any_sync(kFull, (mn[0] > m[0]) || (mn[1] > m[1]))) {
-            float alpha[2];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                alpha[t] = (mn[t] > m[t]) ? fast_exp2(m[t] - mn[t]) : 1.0f;
-                l[t] *= alpha[t];
-                Z[t] *= alpha[t];
-                m[t] = mn[t];
-            }
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const float a0 = __shfl_sync(kFull, alpha[t], 8 * pq);      // row 8 t + 2 pq
-                const float a1 = __shfl_sync(kFull, alpha[t], 8 * pq + 4);  // row 8 t + 2 pq + 1
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    O[t][j][0] *= a0;
-                    O[t][j][1] *= a1;
-                    O[t][j][2] *= a0;
-                    O[t][j][3] *= a1;
-                }
-            }
-        }
-        float pv[2][2][2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
+        // Scores, online softmax and weights; a chunk below every row's length and on valid
+        // pages (FULL, the common case) takes no per-token test.
+        uint32_t bh[2][2], bl[2][2];  // P.V B operands per row half: fp16 high / low parts
+        auto softmax = [&](auto full_c) {
+            constexpr bool FULL = decltype(full_c)::value;
+            float sc[2][2][2];  // [row half][tau][column 2 pq + e]
 #pragma unroll
             for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int lt = 8 * tau + (e ? tokB : tokA);
-                    float pr;
-                    float2 vz;
-                    if (full) {
-                        pr = fast_exp2(sc[t][tau][e] - m[t]);
-                        vz = R.szf[warp][1][lt];
-                    } else {
-                        // masked tokens (past a row's end, skipped pages, stale slots) may hold any
-                        // bits in their scale/zero word: never let them reach an operand, even times 0
-                        const bool live = sc[t][tau][e] != -INFINITY;
-                        pr = live ? fast_exp2(sc[t][tau][e] - m[t]) : 0.0f;
-                        vz = live ? R.szf[warp][1][lt] : make_float2(0.0f, 0.0f);
+                    const float2 kz = R.szf[warp][0][lt];
+                    const float c0 = q_dot(X[tau][e], X[tau][2 + e], W[tau][e]);
+                    const float c1 = q_dot(Y[tau][e], Y[tau][2 + e], W[tau][2 + e]);
+                    sc[0][tau][e] = qsc[0] * fmaf(kz.x, c0, kz.y * qsn[0]);
+                    sc[1][tau][e] = qsc[1] * fmaf(kz.x, c1, kz.y * qsn[1]);
+                    if (!FULL) {
+                        const bool page_ok = ((vmask >> lt) & 1u) != 0;
+                        if (!(page_ok && tb + lt < len[0])) sc[0][tau][e] = -INFINITY;
+                        if (!(page_ok && tb + lt < len[1])) sc[1][tau][e] = -INFINITY;
                     }
-                    l[t] += pr;
-                    Z[t] = fmaf(pr, vz.y, Z[t]);
-                    pv[t][tau][e] = pr * vz.x;
                 }
-        // B operands per row half: (tokA, tokB) of n-tile 0 and 1, fp16 high and low parts
-        uint32_t bh[2][2], bl[2][2];
+            // online softmax (log2 domain) per row; a row's 16 scores sit in one lane quad
+            float mn[2];
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int tau = 0; tau < 2; ++tau) {
-                bh[t][tau] = pack_half2(pv[t][tau][0], pv[t][tau][1]);
-                bl[t][tau] = pack_half2(pv[t][tau][0] - half_lo(bh[t][tau]), pv[t][tau][1] - half_hi(bh[t][tau]));
+            for (int t = 0; t < 2; ++t) {
+                float cm = fmaxf(fmaxf(sc[t][0][0], sc[t][0][1]), fmaxf(sc[t][1][0], sc[t][1][1]));
+                cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 1));
+                cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 2));
+                mn[t] = fmaxf(m[t], cm);
             }
+            if (__any_sync(kFull, (mn[0] > m[0]) || (mn[1] > m[1]))) {
+                float alpha[2];
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    alpha[t] = (mn[t] > m[t]) ? fast_exp2(m[t] - mn[t]) : 1.0f;
+                    l[t] *= alpha[t];
+                    Z[t] *= alpha[t];
+                    m[t] = mn[t];
+                }
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const float a0 = __shfl_sync(kFull, alpha[t], 8 * pq);      // row 8 t + 2 pq
+                    const float a1 = __shfl_sync(kFull, alpha[t], 8 * pq + 4);  // row 8 t + 2 pq + 1
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        O[t][j][0] *= a0;
+                        O[t][j][1] *= a1;
+                        O[t][j][2] *= a0;
+                        O[t][j][3] *= a1;
+                    }
+                }
+            }
+            float pv[2][2][2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int lt = 8 * tau + (e ? tokB : tokA);
+                        float pr;
+                        float2 vz;
+                        if (FULL) {
+                            pr = fast_exp2(sc[t][tau][e] - m[t]);
+                            vz = R.szf[warp][1][lt];
+                        } else {
+                            // masked tokens (past a row's end, skipped pages, stale slots) may hold
+                            // any bits in their scale/zero word: never let them reach an operand,
+                            // even times 0
+                            const bool live = sc[t][tau][e] != -INFINITY;
+                            pr = live ? fast_exp2(sc[t][tau][e] - m[t]) : 0.0f;
+                            vz = live ? R.szf[warp][1][lt] : make_float2(0.0f, 0.0f);
+                        }
+                        l[t] += pr;
+                        Z[t] = fmaf(pr, vz.y, Z[t]);
+                        pv[t][tau][e] = pr * vz.x;
+                    }
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int tau = 0; tau < 2; ++tau) {
+                    bh[t][tau] = pack_half2(pv[t][tau][0], pv[t][tau][1]);
+                    bl[t][tau] =
+                        pack_half2(pv[t][tau][0] - half_lo(bh[t][tau]), pv[t][tau][1] - half_hi(bh[t][tau]));
+                }
+        };
+        if ((tb + kChunk <= tmin) && (vmask == 0xFFFFu))
+            softmax(std::true_type{});
+        else
+            softmax(std::false_type{});
         v_tiles<CB>(st, gq, tokA, tokB, [&](int jv, const uint32_t(&a)[4]) {
             mma16816(O[0][jv], a, bh[0][0], bh[0][1]);
-            mma16816(O[0][jv], a, bl[0][0], bl[0][1]);
             mma16816(O[1][jv], a, bh[1][0], bh[1][1]);
+            mma16816(O[0][jv], a, bl[0][0], bl[0][1]);
             mma16816(O[1][jv], a, bl[1][0], bl[1][1]);
         });
         if ((i % kFoldEvery) == kFoldEvery - 1) fold_acc();

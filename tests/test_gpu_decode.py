@@ -114,3 +114,47 @@ def test_decode_page_sizes(ps):
     for mode, b, rv in ((kvq.KV_INT4_BDR, 128, True), (kvq.KV_INT4, 0, False), (kvq.KV_BF16, 0, False)):
         c = make_case(mode, b, rv, lengths, wl, seed=ps)
         _run(c, lengths)
+
+
+def test_stale_workspace_and_graph_replay():
+    """The split-K scratch needs no initial contents: a workspace full of stale bytes of any
+    kind, repeated calls, and replays of a captured CUDA graph of the decode (split and merge
+    kernels, programmatic dependent launch) all give the same rows as a fresh call."""
+    lengths = [700, 0, 1301, 64, 4100]
+    c = make_case(kvq.KV_INT4_BDR, 128, True, lengths, synth.WORKLOADS["batch16"], seed=41)
+    assert gpu_append(c) == kvq.KV_OK
+    oracle_append(c)
+    assert_pools_equal(c)
+    q = synth.make_q(len(lengths), 32, 128, seed=42).cuda()
+    sl = torch.as_tensor(lengths, dtype=torch.int32).cuda()
+    pt = c.page_table.cuda()
+    ws, n = c.cache.workspace(len(lengths), max(lengths))
+    ref, _ = oracle_decode(c, q.cpu(), lengths)
+    outs = []
+    for fill in (0xFF, 0x00, 0x5A):  # NaN, zero and arbitrary scratch words
+        ws.fill_(fill)
+        outs.append(c.cache.decode(q, sl, pt, max(lengths), out_fp32=True, workspace=(ws, n)))
+        assert c.cache.get_error() == kvq.KV_OK
+    for o in outs:
+        assert torch.equal(o, outs[0])
+    assert attn_rel_err(outs[0].cpu().numpy(), ref) <= ATTN_RTOL
+    assert not outs[0][1].any()  # the empty sequence
+    # capture one decode call in a graph and replay it (its call tag is baked in)
+    out = torch.full_like(outs[0], 3.0)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        kvq.kv_decode_attn(c.cache.handle, q, sl, pt, pt.shape[1], len(lengths), max(lengths), out, 1, ws, n, stream)
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        kvq.kv_decode_attn(c.cache.handle, q, sl, pt, pt.shape[1], len(lengths), max(lengths), out, 1, ws, n,
+                           torch.cuda.current_stream())
+    for _ in range(3):
+        out.fill_(3.0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, outs[0])
+    del g
+    assert c.cache.get_error() == kvq.KV_OK
