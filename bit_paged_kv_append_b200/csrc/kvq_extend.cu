@@ -61,7 +61,7 @@ static_assert(kRows * kHeadDim * 4 <= kStages * kStageBytes, "output rows are st
 __device__ __forceinline__ int ob_idx(int r, int d) { return r * kHeadDim + 4 * ((d >> 2) ^ ((r >> 1) & 3)) + (d & 3); }
 
 template <int G, int CB>
-__global__ void __launch_bounds__(kThreads, 2) extend_kernel(ExtendParams ep) {
+__global__ void __launch_bounds__(kThreads, 3) extend_kernel(ExtendParams ep) {
     static_assert(kRows % G == 0, "a warp holds whole query groups");
     constexpr int QW = kRows / G;   // queries per warp
     constexpr int QB = kWarps * QW;  // queries per CTA
