@@ -447,11 +447,16 @@ def run_e2e(w: Workload, mode, b, rv, steps, warmup, device):
 # --------------------------------------------------------------------------- oracle (CPU)
 
 def oracle_unit_costs(w: Workload, mode, b, rv, tok_budget: int, row_budget: int, seed=0, dec_seqs: int = 1,
-                      reps: int = 1):
+                      reps: int = 1, threads: int = 1):
     """Seconds per appended token and per (cached token x query head) of the CPU oracle, measured
     on a bounded sample shaped like the workload: tok_budget appended tokens, and row_budget
     query-head rows of each of dec_seqs sequences of the workload's mean decoded length; the
-    whole sample is run reps times (seeds seed .. seed + reps - 1) and the times summed."""
+    whole sample is run reps times (seeds seed .. seed + reps - 1) and the times summed.  With
+    threads > 1 the appended tokens and the decoded rows are split into that many contiguous
+    parts run concurrently (the C oracle keeps no global state and ctypes releases the GIL), and
+    the wall time is what counts."""
+    import concurrent.futures
+
     import oracle
 
     H, ps = w.H, w.ps
@@ -461,6 +466,7 @@ def oracle_unit_costs(w: Workload, mode, b, rv, tok_budget: int, row_budget: int
     r = max(1, min(row_budget, w.Hq))
     nd = max(1, dec_seqs)
     t_app = t_dec = 0.0
+    pool = concurrent.futures.ThreadPoolExecutor(max_workers=threads) if threads > 1 else None
     for rep in range(reps):
         sd = seed + rep
         k, v = synth.make_kv(n, w.wl, sd)
@@ -473,20 +479,58 @@ def oracle_unit_costs(w: Workload, mode, b, rv, tok_budget: int, row_budget: int
             ks = np.zeros((P, H, ps, 2), np.uint16)
         vp, vs = kp.copy(), ks.copy()
         ts, tp = synth.append_positions([n])
+        kb, vb, tsn, tpn, ptn = bits(k), bits(v), ts.numpy(), tp.numpy(), pt.numpy()
+        cuts = np.linspace(0, n, max(1, threads) + 1).astype(int)
+
+        def app(part):
+            a, z = cuts[part], cuts[part + 1]
+            oracle.append(mode, b, rv, kp, vp, ks, vs, kb[a:z], vb[a:z], tsn[a:z], tpn[a:z], ptn)
+
         t0 = time.perf_counter()
-        oracle.append(mode, b, rv, kp, vp, ks, vs, bits(k), bits(v), ts.numpy(), tp.numpy(), pt.numpy())
+        if pool:
+            list(pool.map(app, range(threads)))
+        else:
+            app(0)
         t_app += time.perf_counter() - t0
-        q = synth.make_q(nd, w.Hq, 128, sd)
+        qb = bits(synth.make_q(nd, w.Hq, 128, sd))
         rows = [(s, j) for s in range(nd) for j in range(r)]
+        rcuts = np.linspace(0, len(rows), max(1, threads) + 1).astype(int)
+
+        def dec(part):
+            sub = rows[rcuts[part]:rcuts[part + 1]]
+            if sub:
+                oracle.decode(mode, b, rv, kp, vp, ks, vs, qb, np.array([Ls] * nd), ptn, H, rows=sub)
+
         t0 = time.perf_counter()
-        oracle.decode(mode, b, rv, kp, vp, ks, vs, bits(q), np.array([Ls] * nd), pt.numpy(), H, rows=rows)
+        if pool:
+            list(pool.map(dec, range(threads)))
+        else:
+            dec(0)
         t_dec += time.perf_counter() - t0
+    if pool:
+        pool.shutdown()
     c_app = t_app / (n * reps)
     c_dec = t_dec / (r * nd * Ls * reps)
     sample = (f"{reps} x (oracle append of {n} tokens and decode of {r} query-head rows of {nd} sequence(s) "
-              f"over {Ls} cached tokens), 1 thread, {t_app + t_dec:.1f} s; per-unit costs scaled to one step "
-              f"({w.tokens_per_step} tokens appended, {sum(w.dec_lens) * w.Hq} (token x query head) decoded)")
+              f"over {Ls} cached tokens), {threads} thread(s), {t_app + t_dec:.1f} s wall; per-unit costs scaled "
+              f"to one step ({w.tokens_per_step} tokens appended, {sum(w.dec_lens) * w.Hq} (token x query head) "
+              f"decoded)")
     return c_app, c_dec, sample
+
+
+def host_cpu():
+    """(usable cores, CPU model) of this host."""
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return cores, model
 
 
 def oracle_step_seconds(w: Workload, c_app, c_dec):
@@ -645,13 +689,20 @@ def main():
                             "metric": "per (sequence, query head) row max|o-r|/max|r|", **accuracy}
     if rank == 0 and world == 1 and not args.no_cpu:
         # about one step's worth of oracle work per repetition for batch16 (~4 s), bounded for the
-        # large workloads; 3 repetitions: ~10-15 s of host CPU
+        # large workloads; 3 repetitions: ~10-15 s of host CPU on one core, then the same sample
+        # split over every core
         Ls = int(min(max(np.mean(w.dec_lens), 16), 32768))
         nd = max(1, min(w.dec_B, 16, (1 << 20) // (w.Hq * Ls)))
-        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=min(w.tokens_per_step, 40960),
-                                                 row_budget=w.Hq, dec_seqs=nd, reps=3)
+        kw = dict(tok_budget=min(w.tokens_per_step, 40960), row_budget=w.Hq, dec_seqs=nd, reps=3)
+        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, **kw)
+        cores, model = host_cpu()
         line["cpu_baseline"] = {"value": w.tokens_per_step / oracle_step_seconds(w, c_app, c_dec),
-                                "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
+                                "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample,
+                                "cpu_model": model, "host_cores": cores}
+        if cores > 1:
+            p_app, p_dec, psample = oracle_unit_costs(w, hmode, hb, hrv, threads=cores, **kw)
+            line["cpu_baseline"]["all_cores"] = {"value": w.tokens_per_step / oracle_step_seconds(w, p_app, p_dec),
+                                                 "unit": "tokens/s", "cores": cores, "sample": psample}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if _dist is not None:
@@ -660,10 +711,12 @@ def main():
 
 def run_reference(args, world):
     """The CPU oracle as the reference arm (rank 0 only): each step runs a bounded sample of the
-    workload's step on the host cores and scales its unit costs to the full step."""
+    workload's step on all the host's cores (its tokens and rows split over threads) and scales
+    its unit costs to the full step."""
     w = Workload(args.workload, args.seed, torch.device("cpu"))
     _, hmode, hb, hrv = HEADLINE[args.workload]
     budget_s = 120.0
+    cores, model = host_cpu()
     c_app, c_dec, _ = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=256, row_budget=1)
     unit = max(oracle_step_seconds(w, c_app, c_dec), 1e-9)
     frac = min(1.0, budget_s / (args.steps + args.warmup) / unit)
@@ -671,7 +724,8 @@ def run_reference(args, world):
     rows = max(1, int(8 * frac))
     times, sample = [], ""
     for i in range(args.warmup + args.steps):
-        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=tok, row_budget=rows, seed=i)
+        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=tok, row_budget=rows, seed=i,
+                                                 threads=cores)
         if i >= args.warmup:
             times.append(oracle_step_seconds(w, c_app, c_dec))
     step_s = float(np.mean(times))
@@ -681,7 +735,8 @@ def run_reference(args, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32 write path, f64 attention", "data": "synthetic",
             "config": {"workload": args.workload, "variant": HEADLINE[args.workload][0],
                        "sequences": len(w.lengths), "tokens_appended_per_step": w.tokens_per_step},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+                             "cpu_model": model},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
