@@ -139,8 +139,7 @@ kv_status kv_extend_attn(kv_cache* c, const void* q, const int32_t* q_indptr, co
         !aligned(out, 16))
         return KV_ERR_INVALID;
     if (c->g.mode == KV_BF16) return KV_ERR_UNSUPPORTED;
-    const int qb = kvq::extend_queries_per_cta(c->g);
-    if (batch > 65535 || (max_q_len + qb - 1) / qb > 65535) return KV_ERR_UNSUPPORTED;  // grid extents
+    if (batch > 65535) return KV_ERR_UNSUPPORTED;  // the grid's z extent
     kvq::ExtendArgs a{q, q_indptr, seq_lens, page_table, pt_stride, batch, max_q_len, max_seq_len, out,
                       out_fp32 ? 1 : 0};
     cudaError_t e = kvq::launch_extend(c->g, a, c->err_dev, static_cast<cudaStream_t>(stream));

@@ -15,7 +15,8 @@
 // walks every 16-token chunk up to its last query's position with its own ring of
 // chunk stages and online-softmax state, so warps never wait on one another.  Blocks
 // are numbered from each sequence's last query backwards, so the longest rows start
-// first.
+// first, and the query block is the grid's fastest index: the CTAs in flight at any time
+// belong to few (sequence, KV head) pairs, whose codes then stay in L2 for all of them.
 //   * q.K: D[16 rows x 8 tokens] += A[16 x 32 dims] B[32 dims x 8 tokens] on the int8
 //     tensor path, with q' in 23-bit fixed point as three signed bytes per row (m-tile
 //     0: rows 0..7 high | middle bytes, m-tile 1: rows 8..15, m-tile 2: the low bytes
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(kThreads, 3) extend_kernel(ExtendParams ep) {
     extern __shared__ __align__(128) uint8_t dsm[];
     CtaRing& R = *reinterpret_cast<CtaRing*>(dsm);
     const DecodeParams& p = ep.d;
-    const int h = blockIdx.x, s = blockIdx.y, z = blockIdx.z;
+    const int z = blockIdx.x, h = blockIdx.y, s = blockIdx.z;  // z: query block, from the last
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, pq = lane & 3;
 
@@ -452,7 +453,7 @@ cudaError_t launch_extend(const CacheGeom& g, const ExtendArgs& a, int* err_word
     ep.q_indptr = a.q_indptr;
     ep.max_q_len = a.max_q_len;
     const int qb = extend_queries_per_cta(g);
-    const dim3 grid(g.H, a.batch, (a.max_q_len + qb - 1) / qb);
+    const dim3 grid((a.max_q_len + qb - 1) / qb, g.H, a.batch);
     switch (g.Hq / g.H) {
         case 1: return launch_group<1>(ep, grid, s);
         case 2: return launch_group<2>(ep, grid, s);

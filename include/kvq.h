@@ -198,8 +198,7 @@ kv_status kv_decode_attn_noalloc(kv_cache* cache, const void* q, const int32_t* 
  *  max_q_len   >= every n_s (host bound; sizes the grid), max_seq_len >= every seq_len
  *  out         device [total_q, num_q_heads, head_dim], bf16 (round to nearest even of
  *              the fp32 value) or fp32 (out_fp32 != 0)
- * No workspace; one launch.  KV_BF16 pages: KV_ERR_UNSUPPORTED.  batch > 65535 or
- * max_q_len above 65535 blocks of 64 / G queries: KV_ERR_UNSUPPORTED.  Flagged
+ * No workspace; one launch.  KV_BF16 pages or batch > 65535: KV_ERR_UNSUPPORTED.  Flagged
  * (KV_ERR_OOB via kv_get_error): n_s > max_q_len (the queries before the last
  * max_q_len ones are not computed), p < 0 (n_s > seq_len: zero row), p outside the
  * rotary table (zero row), p + 1 beyond the page table or max_seq_len (clamped as in

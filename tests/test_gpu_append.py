@@ -41,9 +41,11 @@ def test_append_batch16(name, mode, b, rv):
 @pytest.mark.parametrize("H,ps,lengths", [
     (8, 16, [1]), (8, 16, [3, 1, 2]), (8, 1, [5, 9]), (8, 7, [33, 1, 70]), (8, 64, [300]),
     (2, 16, [129, 77]), (1, 16, [600]), (16, 16, [17, 40]), (4, 32, [511]), (32, 8, [9, 10]),
+    (8, 1024, [1500, 3]),
 ])
 def test_append_ragged_shapes(H, ps, lengths):
-    """Ragged tails (rows not a multiple of the 256-row tile), tiny and odd page sizes, other head counts."""
+    """Ragged tails (rows not a multiple of the 224-row tile), tiny, odd and the largest page sizes,
+    other head counts."""
     wl = synth.Workload("t", H, 4 * H if H <= 32 else H, 128, ps, synth.OUTLIERS_X20, "test")
     for mode, b, rv in ((kvq.KV_INT4_BDR, 128, True), (kvq.KV_INT4_BDR, 32, False), (kvq.KV_BF16, 0, False)):
         c = make_case(mode, b, rv, lengths, wl, seed=sum(lengths) + H)

@@ -106,7 +106,7 @@ def test_decode_out_of_range_is_flagged():
     assert st == kvq.KV_ERR_OOB
 
 
-@pytest.mark.parametrize("ps", [1, 7, 24, 32, 48])
+@pytest.mark.parametrize("ps", [1, 7, 24, 32, 48, 1024])
 def test_decode_page_sizes(ps):
     """Page sizes that are not a multiple of 16 take the per-token gather; 32 and 48 the bulk copies."""
     wl = synth.Workload("t", 8, 32, 128, ps, synth.OUTLIERS_X20, "test")
