@@ -655,7 +655,9 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 in, int4 codes + fp16 scale/zero cache, fp32 math", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32",
+        "dtype_detail": "bf16 rows in; fp32 rotation and quantiser; INT4 codes + fp16 scale/zero stored; attention on "
+                        "int8 / fp16 tensor-core tiles with int32 / fp32 accumulation", "data": "synthetic",
         "config": {"workload": args.workload, "description": w.wl.description, "variant": hname,
                    "sequences": len(w.lengths), "tokens_appended_per_step": w.tokens_per_step,
                    "sequences_decoded_per_step": w.dec_B, "cached_tokens_decoded_per_step": sum(w.dec_lens),
@@ -732,7 +734,8 @@ def run_reference(args, world):
     value = w.tokens_per_step / step_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32 write path, f64 attention", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "dtype_detail": "oracle: fp32 write path, float64 attention",
+            "data": "synthetic",
             "config": {"workload": args.workload, "variant": HEADLINE[args.workload][0],
                        "sequences": len(w.lengths), "tokens_appended_per_step": w.tokens_per_step},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
