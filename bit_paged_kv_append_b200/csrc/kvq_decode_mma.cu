@@ -50,6 +50,8 @@
 //   * Which dimension and which token each fragment slot stands for is a fixed
 //     permutation chosen so that every thread reads contiguous bytes and the
 //     shared-memory reads are conflict-free; the output mapping undoes it.
+#include <type_traits>
+
 #include "kvq_mma.cuh"
 
 namespace kvq {
@@ -238,67 +240,74 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
             C[tau][0] = q_dot(D[0], D[2], E[0]);  // head gq, column 2 pq
             C[tau][1] = q_dot(D[1], D[3], E[1]);  // head gq, column 2 pq + 1
         }
-        // A chunk whose 16 tokens all lie before the end and on valid pages needs no
-        // per-token masks (the common case).
-        const bool full = (tb + kChunk <= t1) && (vmask == 0xFFFFu);
-        float sc[2][2];
+        // A chunk whose 16 tokens all lie before the end and on valid pages (FULL, the common
+        // case) needs no per-token masks; the two cases are separate code paths.
+        uint32_t b0, b1, b0l, b1l;
+        auto softmax = [&](auto full_c) {
+            constexpr bool FULL = decltype(full_c)::value;
+            float sc[2][2];
 #pragma unroll
-        for (int tau = 0; tau < 2; ++tau)
+            for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int lt = 8 * tau + (e ? tokB : tokA);
-                const float2 kz = R.szf[warp][0][lt];
-                const float v = qsc * fmaf(kz.x, C[tau][e], kz.y * qsn);
-                const bool valid = gval && (full || ((tb + lt < t1) && ((vmask >> lt) & 1u)));
-                sc[tau][e] = valid ? v : -INFINITY;
-            }
-        // ---- online softmax (log2 domain) for head gq ----
-        float cm = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-        cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 1));
-        cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 2));
-        const float mn = fmaxf(m, cm);
-        if (__any_sync(kFull, mn > m)) {
-            const float alpha = (mn > m) ? fast_exp2(m - mn) : 1.0f;
-            l *= alpha;
-            Z *= alpha;
-            m = mn;
-            const float a0 = __shfl_sync(kFull, alpha, 8 * pq);
-            const float a1 = __shfl_sync(kFull, alpha, 8 * pq + 4);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                O[j][0] *= a0;
-                O[j][1] *= a1;
-                O[j][2] *= a0;
-                O[j][3] *= a1;
-            }
-        }
-        float pt_[2][2];
-#pragma unroll
-        for (int tau = 0; tau < 2; ++tau) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int lt = 8 * tau + (e ? tokB : tokA);
-                float pr;
-                float2 vz;
-                if (full) {  // rows past the group hold m = 0 and scores -inf: weight 0
-                    pr = fast_exp2(sc[tau][e] - m);
-                    vz = R.szf[warp][1][lt];
-                } else {
-                    // masked tokens (past the end, skipped pages, stale slots) may hold any bits
-                    // in their scale/zero word: never let them reach an operand, even times 0
-                    const bool live = sc[tau][e] != -INFINITY;
-                    pr = live ? fast_exp2(sc[tau][e] - m) : 0.0f;
-                    vz = live ? R.szf[warp][1][lt] : make_float2(0.0f, 0.0f);
+                for (int e = 0; e < 2; ++e) {
+                    const int lt = 8 * tau + (e ? tokB : tokA);
+                    const float2 kz = R.szf[warp][0][lt];
+                    const float v = qsc * fmaf(kz.x, C[tau][e], kz.y * qsn);
+                    const bool valid = gval && (FULL || ((tb + lt < t1) && ((vmask >> lt) & 1u)));
+                    sc[tau][e] = valid ? v : -INFINITY;
                 }
-                l += pr;
-                Z += pr * vz.y;
-                pt_[tau][e] = pr * vz.x;
+            // ---- online softmax (log2 domain) for head gq ----
+            float cm = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+            cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 1));
+            cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 2));
+            const float mn = fmaxf(m, cm);
+            if (__any_sync(kFull, mn > m)) {
+                const float alpha = (mn > m) ? fast_exp2(m - mn) : 1.0f;
+                l *= alpha;
+                Z *= alpha;
+                m = mn;
+                const float a0 = __shfl_sync(kFull, alpha, 8 * pq);
+                const float a1 = __shfl_sync(kFull, alpha, 8 * pq + 4);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    O[j][0] *= a0;
+                    O[j][1] *= a1;
+                    O[j][2] *= a0;
+                    O[j][3] *= a1;
+                }
             }
-        }
-        const uint32_t b0 = pack_half2(pt_[0][0], pt_[0][1]);
-        const uint32_t b1 = pack_half2(pt_[1][0], pt_[1][1]);
-        const uint32_t b0l = pack_half2(pt_[0][0] - half_lo(b0), pt_[0][1] - half_hi(b0));
-        const uint32_t b1l = pack_half2(pt_[1][0] - half_lo(b1), pt_[1][1] - half_hi(b1));
+            float pt_[2][2];
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int lt = 8 * tau + (e ? tokB : tokA);
+                    float pr;
+                    float2 vz;
+                    if (FULL) {  // rows past the group hold m = 0 and scores -inf: weight 0
+                        pr = fast_exp2(sc[tau][e] - m);
+                        vz = R.szf[warp][1][lt];
+                    } else {
+                        // masked tokens (past the end, skipped pages, stale slots) may hold any
+                        // bits in their scale/zero word: never let them reach an operand, even times 0
+                        const bool live = sc[tau][e] != -INFINITY;
+                        pr = live ? fast_exp2(sc[tau][e] - m) : 0.0f;
+                        vz = live ? R.szf[warp][1][lt] : make_float2(0.0f, 0.0f);
+                    }
+                    l += pr;
+                    Z += pr * vz.y;
+                    pt_[tau][e] = pr * vz.x;
+                }
+            }
+            b0 = pack_half2(pt_[0][0], pt_[0][1]);
+            b1 = pack_half2(pt_[1][0], pt_[1][1]);
+            b0l = pack_half2(pt_[0][0] - half_lo(b0), pt_[0][1] - half_hi(b0));
+            b1l = pack_half2(pt_[1][0] - half_lo(b1), pt_[1][1] - half_hi(b1));
+        };
+        if ((tb + kChunk <= t1) && (vmask == 0xFFFFu))
+            softmax(std::true_type{});
+        else
+            softmax(std::false_type{});
         pv_chunk<true, CB>(O, st, gq, tokA, tokB, b0, b1, b0l, b1l);
         __syncwarp();  // every lane is done with this slot
         if (i + kStages < nw) cs.issue(p, i + kStages, slot);
