@@ -30,7 +30,7 @@
  *  [WIS4] same blog, section 4 ("experiments"): ablations over key-only versus
  *         key+value rotation and over the block size.
  *
- * Readings where the pages are silent (every one is listed in the design doc):
+ * Readings where the pages are silent:
  *  R1 H_b is Sylvester's Hadamard matrix in natural order,
  *     H[i][j] = (-1)^popcount(i & j), normalised by 1/sqrt(b).
  *  R2 The fp32 FWHT runs its butterfly stages with increasing stride
