@@ -1,0 +1,70 @@
+"""Host-side logic of bench.py (CPU only): the work and byte counts it reports for the extend
+leg, and the all-cores oracle baseline, whose threads must compute exactly what one call does."""
+import concurrent.futures
+
+import numpy as np
+import torch
+
+import bench
+import oracle
+from bit_paged_kv_append_b200 import kvq, synth
+
+
+def test_extend_work_counts_match_the_oracle_positions():
+    """bench counts sum over queries of (position + 1) attended tokens per query head; the oracle's
+    extend_lengths gives every query's position + 1 directly."""
+    for name in ("batch16", "mixed256"):
+        w = bench.Workload(name, 0, torch.device("cpu"))
+        seqs, lens, qlens = bench.extend_setup(w)
+        assert len(seqs) == len(lens) == len(qlens)
+        qi = np.concatenate([[0], np.cumsum(qlens)])
+        _, per_query = oracle.extend_lengths(qi, lens)
+        counted = sum(n * (L - n) + n * (n + 1) // 2 for L, n in zip(lens, qlens))
+        assert counted == int(per_query.sum())
+        assert per_query.min() >= 1  # every query has at least itself to attend to
+        if name == "mixed256":
+            assert qlens == [2048] * 8 and all(L >= 2048 + 1024 for L in lens)
+        else:
+            assert qlens == lens  # a full causal prefill of every sequence
+
+
+def test_threaded_oracle_append_equals_one_call():
+    """The all-cores baseline splits the appended tokens over threads: the pools must come out
+    bit for bit as one call writes them (the oracle keeps no global state)."""
+    wl = synth.WORKLOADS["batch16"]
+    n, H, ps = 3000, wl.num_kv_heads, wl.page_size
+    k, v = synth.make_kv(n, wl, 5)
+    pt, P = synth.make_page_table([n], ps, 5)
+    ts, tp = synth.append_positions([n])
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    kb, vb = bits(k), bits(v)
+
+    def pools():
+        kp = np.zeros((P, H, ps, 64), np.uint8)
+        ks = np.zeros((P, H, ps, 2), np.uint16)
+        return kp, kp.copy(), ks, ks.copy()
+
+    one = pools()
+    oracle.append(oracle.MODE_INT4_BDR, 128, True, *one, kb, vb, ts.numpy(), tp.numpy(), pt.numpy())
+    split = pools()
+    cuts = np.linspace(0, n, 9).astype(int)
+
+    def part(i):
+        a, z = cuts[i], cuts[i + 1]
+        oracle.append(oracle.MODE_INT4_BDR, 128, True, *split, kb[a:z], vb[a:z], ts.numpy()[a:z], tp.numpy()[a:z],
+                      pt.numpy())
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=8) as ex:
+        list(ex.map(part, range(8)))
+    for x, y in zip(one, split):
+        assert np.array_equal(x, y)
+
+
+def test_oracle_unit_costs_threads_and_host_cpu():
+    w = bench.Workload("single256", 0, torch.device("cpu"))
+    for threads in (1, 4):
+        c_app, c_dec, sample = bench.oracle_unit_costs(w, kvq.KV_INT4_BDR, 128, False, tok_budget=256, row_budget=8,
+                                                       threads=threads)
+        assert c_app > 0 and c_dec > 0 and f"{threads} thread(s)" in sample
+    cores, model = bench.host_cpu()
+    assert cores >= 1 and isinstance(model, str) and model
