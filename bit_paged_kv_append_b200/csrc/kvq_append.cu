@@ -143,8 +143,9 @@ __device__ __forceinline__ void rotate_row(float2 (&R)[64], float r_b) {
 }
 
 // Codes of a row into 16 packed words: wa = elements 0..63, wb = elements 64..127.
-// u = fma(y - zero, inv, 1.5 * 2^23) rounds the exact quotient to the nearest
-// integer (ties to even) in its low mantissa bits.  CLAMP maps quotients below 0
+// u = fma(y - zero, inv, 1.5 * 2^23) rounds the exact product fl(y - zero) * inv to the
+// nearest integer (ties to even) in its low mantissa bits: the fma adds the unrounded
+// product to the magic constant and rounds once.  CLAMP maps products below 0
 // (or NaN) to 0 and above 15 to 15; rows whose extreme codes are in range skip it.
 template <bool CLAMP>
 __device__ __forceinline__ void quantise_pack(const float2 (&R)[64], float zf, float inv, uint32_t (&wa)[8],

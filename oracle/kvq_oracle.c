@@ -213,8 +213,10 @@ void oracle_quant_row_bits(const float* y, int D, int bits, uint8_t* codes, uint
     for (int j = 0; j < nbytes; j++) codes[j] = 0;
     for (int e = 0; e < D; e++) {
         float t = y[e] - zero;
-        /* the quotient t * inv is rounded to an integer from its exact value: the
-         * product of two floats is exact in double (24 + 24 < 53 significant bits) */
+        /* R4: rint (ties to even) of the exact product fl(y - zero) * fl(1/scale),
+         * one rounding straight to an integer (not the product rounded to fp32 first,
+         * and not the exact quotient (y - zero) / scale).  The product of two floats is
+         * exact in double (24 + 24 < 53 significant bits). */
         double v = (double)t * (double)inv;
         double r = rint(v); /* default rounding mode: nearest, ties to even */
         int code;

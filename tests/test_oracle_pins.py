@@ -20,6 +20,7 @@ import oracle
 from bit_paged_kv_append_b200 import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 BLOCKS = [2, 4, 8, 16, 32, 64, 128]
 
 
@@ -165,17 +166,77 @@ def _row_d():
     return y
 
 
-@pytest.mark.parametrize("row", ["A", "B", "C", "D"])
+def _row_e():
+    y = np.zeros(128)
+    y[1], y[2], y[3], y[4] = 1.5, 15934463 / 2 ** 24, 7371 / 2 ** 14, 23751 / 2 ** 14
+    return y
+
+
+def _worked_row(row):
+    i = np.arange(128)
+    return {"A": 0.5 * (i % 16), "B": -3 + 0.25 * (i % 16), "C": np.full(128, 1.75), "D": _row_d(),
+            "E": _row_e()}[row].astype(np.float32)
+
+
+@pytest.mark.parametrize("row", ["A", "B", "C", "D", "E"])
 def test_quant_worked_examples(row):
     g = _golden()
-    i = np.arange(128)
-    y = {"A": 0.5 * (i % 16), "B": -3 + 0.25 * (i % 16), "C": np.full(128, 1.75), "D": _row_d()}[row].astype(
-        np.float32)
-    codes, sz = oracle.quant_row(y)
+    codes, sz = oracle.quant_row(_worked_row(row))
     assert sz[0] == int(g[f"{row}.scale"][0], 16)
     assert sz[1] == int(g[f"{row}.zero"][0], 16)
     want = bytes.fromhex("".join(g[f"{row}.bytes"]))
     assert codes.tobytes() == want
+
+
+# The rounding step of the oracle's quantiser, as written in kvq_oracle.c, and the two
+# other readings of "round to nearest" that the worked rows D and E tell apart: the
+# product rounded to fp32 before the rounding to an integer, and the exact quotient.
+_R4_LINE = "double v = (double)t * (double)inv;"
+_R4_MUTANTS = {"fp32_product": "double v = (double)(float)(t * inv);",
+               "exact_quotient": "double v = (scale > 0.0f) ? (double)t / (double)scale : 0.0;"}
+
+
+def _mutant_quant_row(tmp_path, name):
+    """oracle_quant_row from a copy of the oracle whose rounding step is replaced by another
+    reading (a planted mistake, built and run on the CPU only)."""
+    import ctypes
+    import subprocess
+
+    src = open(os.path.join(ROOT, "oracle", "kvq_oracle.c")).read()
+    assert src.count(_R4_LINE) == 1, "the oracle's rounding step moved; update the mutants"
+    path = tmp_path / f"oracle_{name}.c"
+    path.write_text(src.replace(_R4_LINE, _R4_MUTANTS[name]))
+    lib_path = tmp_path / f"liboracle_{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=gnu11", "-shared", "-fPIC",
+                           "-o", str(lib_path), str(path), "-lm"])
+    lib = ctypes.CDLL(str(lib_path))
+    P = ctypes.c_void_p
+    lib.oracle_quant_row.argtypes = [P, ctypes.c_int, P, P]
+
+    def quant_row(y):
+        y = np.ascontiguousarray(y, dtype=np.float32)
+        codes = np.zeros(64, np.uint8)
+        sz = np.zeros(2, np.uint16)
+        lib.oracle_quant_row(y.ctypes.data_as(P), 128, codes.ctypes.data_as(P), sz.ctypes.data_as(P))
+        return codes, sz
+
+    return quant_row
+
+
+@pytest.mark.parametrize("name", sorted(_R4_MUTANTS))
+def test_worked_rows_reject_the_other_rounding_readings(tmp_path, name):
+    """Rows D and E pin the rounding reading: an oracle built with either other reading
+    computes different bytes for both rows (and row E's bytes are the ones derived by hand
+    for that reading in the golden file)."""
+    g = _golden()
+    quant_row = _mutant_quant_row(tmp_path, name)
+    for row in ("D", "E"):
+        codes, sz = quant_row(_worked_row(row))
+        assert sz[0] == int(g[f"{row}.scale"][0], 16) and sz[1] == int(g[f"{row}.zero"][0], 16)
+        assert codes.tobytes() != bytes.fromhex("".join(g[f"{row}.bytes"])), row
+    codes, _ = quant_row(_worked_row("E"))
+    key = {"fp32_product": "E.bytes_if_fp32_product", "exact_quotient": "E.bytes_if_exact_quotient"}[name]
+    assert codes.tobytes() == bytes.fromhex("".join(g[key]))
 
 
 def test_pack_unpack_all_byte_values():
@@ -209,9 +270,11 @@ def test_quant_error_bound_and_monotone(mag):
         assert np.all(np.diff(c[order].astype(int)) >= 0)
 
 
-def test_quant_rounds_the_exact_quotient():
-    """The code is the integer nearest the exact product fl(y - zero) * fl(1/scale) (ties to
-    even), checked with rational arithmetic on random rows."""
+def test_quant_cross_check_exact_product_on_random_rows():
+    """Cross-check, not a pin: it restates the oracle's rounding step (rint, ties to even, of
+    the exact product fl(y - zero) * fl(1/scale)) with rational arithmetic on random rows, so
+    it only confirms that the C code computes what it says.  The pins of that step are the
+    hand-derived rows D and E above."""
     from fractions import Fraction
 
     rng = np.random.default_rng(17)
