@@ -10,13 +10,6 @@
 #include "kvq.h"
 #include "kvq_internal.h"
 
-struct kv_cache {
-    kvq::CacheGeom g;
-    int* err_dev;  // device error word (bit flags, see kvq_common.cuh)
-    int device;
-    int num_sms;
-};
-
 namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -104,6 +97,8 @@ kv_status kv_append_quant(kv_cache* c, const void* k, const void* v, int num_tok
         return KV_ERR_INVALID;
     if (pt_stride < 1 || num_seqs < 1) return KV_ERR_INVALID;
     kvq::AppendArgs a{k, v, num_tokens, tok_seq, tok_pos, page_table, pt_stride, num_seqs};
+    kvq::DeviceGuard dg(c->device);
+    if (!dg.ok()) return KV_ERR_CUDA;
     cudaError_t e = kvq::launch_append(c->g, a, c->err_dev, c->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
@@ -125,6 +120,8 @@ kv_status kv_decode_attn(kv_cache* c, const void* q, const int32_t* seq_lens, co
     if (!workspace || workspace_bytes < plan.ws_bytes || !aligned(workspace, 16)) return KV_ERR_INVALID;
     kvq::DecodeArgs a{q, seq_lens, page_table, pt_stride, batch, max_seq_len, out, out_fp32 ? 1 : 0,
                       workspace, workspace_bytes};
+    kvq::DeviceGuard dg(c->device);
+    if (!dg.ok()) return KV_ERR_CUDA;
     cudaError_t e = kvq::launch_decode(c->g, a, plan, c->err_dev, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
@@ -142,6 +139,8 @@ kv_status kv_extend_attn(kv_cache* c, const void* q, const int32_t* q_indptr, co
     if (batch > 65535) return KV_ERR_UNSUPPORTED;  // the grid's z extent
     kvq::ExtendArgs a{q, q_indptr, seq_lens, page_table, pt_stride, batch, max_q_len, max_seq_len, out,
                       out_fp32 ? 1 : 0};
+    kvq::DeviceGuard dg(c->device);
+    if (!dg.ok()) return KV_ERR_CUDA;
     cudaError_t e = kvq::launch_extend(c->g, a, c->err_dev, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
@@ -149,6 +148,8 @@ kv_status kv_extend_attn(kv_cache* c, const void* q, const int32_t* q_indptr, co
 kv_status kv_get_error(kv_cache* c, void* stream) {
     if (!c) return KV_ERR_INVALID;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    kvq::DeviceGuard dg(c->device);
+    if (!dg.ok()) return KV_ERR_CUDA;
     int h = 0;
     if (cudaStreamSynchronize(s) != cudaSuccess) return KV_ERR_CUDA;
     if (cudaMemcpyAsync(&h, c->err_dev, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
@@ -161,7 +162,10 @@ kv_status kv_get_error(kv_cache* c, void* stream) {
 
 void kv_free(kv_cache* c) {
     if (!c) return;
-    cudaFree(c->err_dev);
+    {
+        kvq::DeviceGuard dg(c->device);
+        cudaFree(c->err_dev);
+    }
     delete c;
 }
 

@@ -45,7 +45,7 @@ constexpr int kStageBytes = 2 * kHalfBytes;  // 56 KiB (a multiple of 1 KiB: swi
 constexpr int kMaxTileTokens = kRows;        // H == 1
 constexpr size_t kSmemBytes = 1024 /*align slack*/ + size_t(kStages) * kStageBytes +
                               2 * size_t(kMaxTileTokens) * (sizeof(int2) + sizeof(int)) +
-                              2 * kStages * sizeof(uint64_t);
+                              2 * kStages * sizeof(uint64_t) + 16 /*abort flag*/;
 
 // Magic constant 1.5 * 2^23: for |v| < 2^22, the fp32 sum v + kMagic (rounded to
 // nearest even) carries rint_even(v) in its low mantissa bits.
@@ -357,6 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* mpos = reinterpret_cast<int*>(meta + 2 * kMaxTileTokens);       // [tile parity][tile token] = position
     uint64_t* full = reinterpret_cast<uint64_t*>(mpos + 2 * kMaxTileTokens);
     uint64_t* empty = full + kStages;
+    // set by the producer when it gives up a wait: a stage released after that carries no
+    // tile and its consumers leave without reading it
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -367,6 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full[e], 1);
             mbar_init(&empty[e], kRows / 32);
         }
+        *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
@@ -391,6 +395,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 b[r] = in ? __ldg(p.a.tok_pos + t) : -1;
             }
         };
+        // Before the warp leaves: every stage copy it issued (issued = fills so far) has
+        // landed, waited for with the usual bound, so the CTA never exits while a bulk copy
+        // into its shared memory is in flight.
+        auto drain = [&](int issued) {
+            for (int e = 0; e < kStages; ++e) {
+                if (issued > e && !mbar_wait(&full[e], ((issued - 1 - e) / kStages) & 1))
+                    flag_error(p.err, kErrTimeout);
+            }
+        };
         load_ids(blockIdx.x, sq, po);
         int seqno = 0, n = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++n) {
@@ -403,6 +416,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 es[kv] = e;
                 if (fill > 0 && !mbar_wait(&empty[e], (fill - 1) & 1)) {
                     flag_error(p.err, kErrTimeout);
+                    // release the K stage this tile already filled (its arrival completes the
+                    // phase; the flag tells its consumers to skip it), then drain and leave
+                    if (lane == 0) {
+                        *abort_flag = 1;
+                        if (kv == 1) mbar_arrive(&full[es[0]]);
+                    }
+                    __syncwarp();
+                    drain(seqno);
                     return;
                 }
                 if (lane == 0) {
@@ -448,6 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 po[r] = npo[r];
             }
         }
+        drain(seqno);
         return;
     }
 
@@ -463,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 flag_error(p.err, kErrTimeout);
                 return;
             }
+            if (*abort_flag) return;  // the producer gave up: this stage holds no tile
             if (kv == 0) m = meta[(n & 1) * kMaxTileTokens + tt];
             // key rows turn at the token's position (the position was checked by the producer)
             const float* cs = (ROPE && kv == 0 && m.x >= 0)
@@ -521,13 +544,9 @@ bool make_row_map(CUtensorMap* map, const void* base, int64_t rows) {
 
 template <int MODE, int BLK, bool ROTV, bool ROPE, int CB>
 cudaError_t launch_r(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
-    auto kern = append_kernel<MODE, BLK, ROTV, ROPE, CB>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    constexpr auto kern = append_kernel<MODE, BLK, ROTV, ROPE, CB>;
+    const cudaError_t e = ensure_smem_opt_in<kern>(kSmemBytes);
+    if (e != cudaSuccess) return e;
     return launch_overlapped(kern, dim3(grid), dim3(kThreads), kSmemBytes, s, km, vm, p);
 }
 

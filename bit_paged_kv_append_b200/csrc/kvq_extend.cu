@@ -416,13 +416,9 @@ __global__ void __launch_bounds__(kThreads, 3) extend_kernel(ExtendParams ep) {
 
 template <int G, int CB>
 cudaError_t launch_k(const ExtendParams& ep, dim3 grid, cudaStream_t s) {
-    auto kern = extend_kernel<G, CB>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    constexpr auto kern = extend_kernel<G, CB>;
+    const cudaError_t e = ensure_smem_opt_in<kern>(kSmemBytes);
+    if (e != cudaSuccess) return e;
     return launch_overlapped(kern, grid, dim3(kThreads), kSmemBytes, s, ep);
 }
 

@@ -78,4 +78,38 @@ cudaError_t launch_extend(const CacheGeom& g, const ExtendArgs& a, int* err_word
 // Query rows one extend CTA covers for this cache (grid extent along the queries: max_q_len / this).
 int extend_queries_per_cta(const CacheGeom& g);
 
+// Makes the handle's device current for the duration of one C-ABI call (and restores the
+// caller's device afterwards), so that launches, function attributes and symbol lookups
+// all refer to the device the cache's pools live on.
+class DeviceGuard {
+  public:
+    explicit DeviceGuard(int device) : prev_(-1) {
+        int cur = -1;
+        ok_ = cudaGetDevice(&cur) == cudaSuccess;
+        if (ok_ && cur != device) {
+            ok_ = cudaSetDevice(device) == cudaSuccess;
+            if (ok_) prev_ = cur;
+        }
+    }
+    ~DeviceGuard() {
+        if (prev_ >= 0) cudaSetDevice(prev_);
+    }
+    bool ok() const { return ok_; }
+    DeviceGuard(const DeviceGuard&) = delete;
+    DeviceGuard& operator=(const DeviceGuard&) = delete;
+
+  private:
+    int prev_;
+    bool ok_;
+};
+
 }  // namespace kvq
+
+// The opaque handle of include/kvq.h (the only definition: kvq_api.cu and kvq_noalloc.cu
+// both use this one).
+struct kv_cache {
+    kvq::CacheGeom g;
+    int* err_dev;  // device error word (bit flags, see kvq_common.cuh)
+    int device;    // the device current at kv_create_paged: every call runs there
+    int num_sms;
+};

@@ -13,7 +13,8 @@
 // (KV_NOALLOC_SCRATCH_BYTES in kvq.h).  Every GPU that loads this library
 // holds it until the process exits.  In host code the array's name is only a
 // host-side stand-in, so its device address is obtained once per device with
-// cudaGetSymbolAddress (on the first call made while that device is current)
+// cudaGetSymbolAddress (on the first call for a handle on that device, which the call
+// makes current while it runs)
 // and then passed to the kernels like any workspace pointer.  Nothing in the
 // scratch has to start at zero: the split kernel writes every partial result
 // the merge kernel reads, on every call.  All calls share the one array, so
@@ -27,13 +28,6 @@
 #include "kvq.h"
 #include "kvq_internal.h"
 
-struct kv_cache {  // same layout as the definition in kvq_api.cu
-    kvq::CacheGeom g;
-    int* err_dev;
-    int device;
-    int num_sms;
-};
-
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = KV_NOALLOC_SCRATCH_BYTES;
@@ -45,8 +39,8 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_decode_scratch on the current device (looked up once per
-// device); nullptr on failure.
+// Device address of g_decode_scratch on `device`, which must be current (looked up once
+// per device, under a lock); nullptr on failure.
 void* scratch_address(int device) {
     if (device < 0 || device >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
@@ -72,9 +66,10 @@ extern "C" kv_status kv_decode_attn_noalloc(kv_cache* c, const void* q, const in
         return KV_ERR_INVALID;
     const kvq::DecodePlan plan = kvq::plan_decode(c->g, batch, max_seq_len, c->num_sms);
     if (plan.ws_bytes > kNoAllocScratchBytes) return KV_ERR_SCRATCH_TOO_SMALL;
-    int device = -1;
-    if (cudaGetDevice(&device) != cudaSuccess) return KV_ERR_CUDA;
-    void* scratch = scratch_address(device);
+    // the handle's device, current while the address is looked up and the kernels launch
+    kvq::DeviceGuard dg(c->device);
+    if (!dg.ok()) return KV_ERR_CUDA;
+    void* scratch = scratch_address(c->device);
     if (!scratch) return KV_ERR_CUDA;
     kvq::DecodeArgs a{q, seq_lens, page_table, pt_stride, batch, max_seq_len, out, out_fp32 ? 1 : 0,
                       scratch, kNoAllocScratchBytes};

@@ -22,7 +22,7 @@ KV_BF16, KV_INT4, KV_INT4_BDR = 0, 1, 2
 HEAD_DIM = 128
 
 EXPORTS = ("kv_create_paged", "kv_append_quant", "kv_decode_workspace_bytes", "kv_decode_attn", "kv_get_error",
-           "kv_free", "kv_status_string", "kv_decode_attn_noalloc")
+           "kv_free", "kv_status_string", "kv_decode_attn_noalloc", "kv_extend_attn")
 
 
 class KVQError(RuntimeError):

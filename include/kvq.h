@@ -44,6 +44,10 @@
  *               page page_table[s * pt_stride + p / page_size], slot
  *               p % page_size.
  *
+ * Devices: a handle belongs to the device that was current when kv_create_paged
+ * made it; every later call on the handle makes that device current while it runs
+ * and restores the caller's device before returning.
+ *
  * Ownership and errors: the library owns only the opaque handle and one
  * device error word.  Every call is asynchronous on the given stream
  * (a cudaStream_t passed as void*, NULL = legacy default stream).  Arguments
@@ -171,9 +175,10 @@ kv_status kv_decode_attn(kv_cache* cache, const void* q, const int32_t* seq_lens
  * call allocates nothing.  Calls whose scratch need,
  * kv_decode_workspace_bytes(cache, batch, max_seq_len), exceeds that size return
  * KV_ERR_SCRATCH_TOO_SMALL before launching anything.
- *  - The first call on a device (with that device current) looks up the array's
- *    device address with cudaGetSymbolAddress; make that first call before any
- *    stream capture on the device.
+ *  - The first call for a handle on a given device looks up the array's device
+ *    address there with cudaGetSymbolAddress (the call makes the handle's device
+ *    current while it runs); make that first call before any stream capture on
+ *    the device.
  *  - Every call shares the one array: calls whose kernels may overlap on the GPU
  *    (different streams, unsynchronised threads) race on it; order them on one
  *    stream.  No part of the array needs to start at zero: each call writes all

@@ -139,6 +139,32 @@ def oracle_decode(c: Case, q, seq_lens, rows=None, page_table=None):
                          code_bits=c.code_bits)
 
 
+def oracle_decode_rows(mode, bdr, rotate_v, pools, q_bits, seq_lens, page_table, num_kv_heads, rows, threads=None,
+                       rope=None, code_bits=4):
+    """oracle.decode over the given (sequence, query head) rows, split into contiguous parts run
+    on concurrent threads (the C oracle keeps no global state and ctypes releases the GIL); the
+    rows come back in the order given.  Returns (out float64 [n, D], skipped-token count)."""
+    import concurrent.futures
+    import os
+
+    kp, vp, ks, vs = pools
+    rows = [tuple(map(int, r)) for r in rows]
+    n = len(rows)
+    threads = max(1, min(threads or (os.cpu_count() or 1), n))
+    cuts = np.linspace(0, n, threads + 1).astype(int)
+
+    def part(i):
+        sub = rows[cuts[i]:cuts[i + 1]]
+        if not sub:
+            return np.zeros((0, 128)), 0
+        return oracle.decode(mode, bdr, rotate_v, kp, vp, ks, vs, q_bits, np.asarray(seq_lens), page_table,
+                             num_kv_heads, rows=sub, rope=rope, code_bits=code_bits)
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        parts = list(ex.map(part, range(threads)))
+    return np.concatenate([p[0] for p in parts]), sum(p[1] for p in parts)
+
+
 def attn_rel_err(got: np.ndarray, ref: np.ndarray) -> float:
     """max over rows of max_i |got - ref| / max_i |ref| (rows with ref == 0 compare absolutely)."""
     got = got.reshape(-1, got.shape[-1]).astype(np.float64)

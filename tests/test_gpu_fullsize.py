@@ -1,15 +1,16 @@
 """Parity at the full sizes of the serving workloads, in the launch configuration bench.py
 times: the whole cache is built with kv_append_quant on the GPU, then a serving step (new
 tokens appended, decode attention) runs; sampled appended rows are compared bit for bit
-with the oracle's quantiser and sampled (sequence, query head) attention rows with the
-oracle's float64 decode over the same pages."""
+with the oracle's quantiser, and every query head of at least two whole sequences (the
+longest among them where lengths differ; the one sequence of long1m) with the oracle's
+float64 decode over the same pages."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from bit_paged_kv_append_b200 import kvq, synth
-from kvq_testlib import ATTN_RTOL, attn_rel_err, bits16
+from kvq_testlib import ATTN_RTOL, attn_rel_err, bits16, oracle_decode_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -47,10 +48,9 @@ def _check_decode(cache, q, seq_lens, pt, max_len, mode, b, rv, rows):
     out16 = cache.decode(q, torch.as_tensor(seq_lens, dtype=torch.int32, device="cuda"), pt, max_len)
     assert cache.get_error() == kvq.KV_OK
     assert torch.equal(out16, out.to(torch.bfloat16))
-    kp, vp = cache.k_pool.cpu().numpy(), cache.v_pool.cpu().numpy()
-    ks, vs = _pool_bits(cache.k_sz), _pool_bits(cache.v_sz)
-    ref, skipped = oracle.decode(mode, b, rv, kp, vp, ks, vs, bits16(q), np.asarray(seq_lens), pt.cpu().numpy(),
-                                 cache.num_kv_heads, rows=rows)
+    pools = (cache.k_pool.cpu().numpy(), cache.v_pool.cpu().numpy(), _pool_bits(cache.k_sz), _pool_bits(cache.v_sz))
+    ref, skipped = oracle_decode_rows(mode, b, rv, pools, bits16(q), seq_lens, pt.cpu().numpy(), cache.num_kv_heads,
+                                      rows)
     assert skipped == 0
     got = np.stack([out[s, j].cpu().numpy() for s, j in rows])
     err = attn_rel_err(got, ref)
@@ -80,7 +80,9 @@ def test_decode64x8k_step():
     _check_rows(cache, k1, v1, ts1.cuda(), tp1.cuda(), pt, mode, b, rv, B, seed=2)
     new_lens = [L + 1 for L in lengths]
     q = synth.make_q(B, Hq, 128, seed=3).cuda()
-    rows = [(s, j) for s, j in zip(np.random.default_rng(4).choice(B, 12), np.random.default_rng(5).choice(Hq, 12))]
+    # every query head of two whole sequences (all lengths are equal here)
+    seqs = [0, int(np.random.default_rng(4).integers(1, B))]
+    rows = [(s, j) for s in seqs for j in range(Hq)]
     _check_decode(cache, q, new_lens, ptd, max(new_lens), mode, b, rv, rows)
 
 
@@ -117,8 +119,10 @@ def test_mixed256_step():
     dl = [lengths[s] + 1 for s in decoding]
     ptdec = pt[decoding].contiguous()
     q = synth.make_q(len(decoding), Hq, 128, seed=4).cuda()
-    rr = np.random.default_rng(8)
-    rows = [(int(s), int(j)) for s, j in zip(rr.choice(len(decoding), 8), rr.choice(Hq, 8))]
+    # every query head of the longest decoding sequence and of one other
+    longest = int(np.argmax(dl))
+    other = int(np.random.default_rng(8).choice([i for i in range(len(decoding)) if i != longest]))
+    rows = [(s, j) for s in (longest, other) for j in range(Hq)]
     _check_decode(cache, q, dl, ptdec.cuda(), max(dl), mode, b, rv, rows)
 
 
@@ -140,4 +144,4 @@ def test_long1m_chunked_append_and_decode():
     _check_rows(cache, k, v, ts, tp, pt, mode, b, rv, 1024, seed=1)
     del k, v
     q = synth.make_q(1, Hq, 128, seed=3).cuda()
-    _check_decode(cache, q, [L], ptd, L, mode, b, rv, [(0, 0), (0, 13), (0, 31)])
+    _check_decode(cache, q, [L], ptd, L, mode, b, rv, [(0, j) for j in range(Hq)])  # every query head

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from bit_paged_kv_append_b200 import kvq, synth
-from kvq_testlib import ATTN_RTOL, attn_rel_err, gpu_append, make_case
+from kvq_testlib import ATTN_RTOL, assert_pools_equal, attn_rel_err, gpu_append, make_case, oracle_append, oracle_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -33,6 +33,8 @@ def test_noalloc_matches_workspace_decode_on_consecutive_calls():
     lengths = synth.seq_lengths("batch16", seed=0)
     c = make_case(kvq.KV_INT4_BDR, 128, True, lengths, wl, seed=0)
     assert gpu_append(c) == kvq.KV_OK
+    oracle_append(c)
+    assert_pools_equal(c)
     # two calls in a row with different queries and batch shapes: the second must not see the first's scratch
     calls = [(synth.make_q(16, 32, 128, seed=11), lengths, max(lengths)),
              (synth.make_q(16, 32, 128, seed=12), [L // 3 for L in lengths], 5000)]
@@ -41,7 +43,12 @@ def test_noalloc_matches_workspace_decode_on_consecutive_calls():
         torch.cuda.synchronize()
         ref = _decode_ws(c, q, lens, max_len)
         assert c.cache.get_error() == kvq.KV_OK
-        assert attn_rel_err(got.cpu().numpy(), ref.cpu().numpy().astype(np.float64)) <= ATTN_RTOL
+        # the same plan and kernels as kv_decode_attn: the same bits
+        assert torch.equal(got, ref)
+        # and within the attention tolerance of the float64 oracle
+        want, skipped = oracle_decode(c, q, lens)
+        assert skipped == 0
+        assert attn_rel_err(got.cpu().numpy(), want) <= ATTN_RTOL
         got16 = _decode_noalloc(c, q, lens, max_len, out_fp32=False)
         assert torch.equal(got16, got.to(torch.bfloat16))
 
