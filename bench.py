@@ -7,17 +7,27 @@ the fused BDR + INT4 appends of the step's new tokens into the paged cache
 merge kernels).  Workloads (synthetic, seeded; K/V ~ N(0,1) with outlier
 channels, q ~ N(0,1)):
 
-  batch16      (default) 16 sequences, lengths ~U[512, 4096], page size 16: a step
-               appends every token of every sequence, then decodes all 16.
+  single256    1 sequence x 256 tokens, page size 16: append it, decode it.
+  batch16      16 sequences, lengths ~U[512, 4096], page size 16: a step appends
+               every token of every sequence, then decodes all 16.
   decode64x8k  64 x 8192 cached tokens (prefilled, untimed): a step appends 1
                token per sequence at position 8192 and decodes 8193 tokens each.
-  mixed256     256 sequences, lengths log-uniform [1024, 32768], 64 query heads,
-               K and V rotated (prefilled, untimed): a step appends a 2048-token
-               chunk to 8 sequences and 1 token to each of the other 248, then
-               decodes those 248.
+  mixed256     (default) 256 sequences, lengths log-uniform [1024, 32768], 64
+               query heads, K and V rotated (prefilled, untimed): a step appends
+               a 2048-token chunk to 8 sequences and 1 token to each of the other
+               248, then decodes those 248.  The largest single-GPU workload with
+               both halves of the path.
   long1m       1 sequence x 1,048,576 tokens, page size 64: a step appends the
                context in 128 chunks of 8192 tokens, then decodes it (split-K).
 Steps rewrite the same slots each time, so every step does the same work.
+
+The headline line times exactly --steps steps of the chosen workload, with CUDA
+events on the launching stream at the start of each step, between its appends and
+its decode, and at its end.  ``value`` is the appended tokens per second of the
+append kernel's own time (the metric's first half); the decode's HBM GB/s is the
+second half.  Unless --no-configs, the line also carries a sub-record per workload
+(all five) with the append and decode rates of INT4+BDR-128, naive INT4 and BF16
+pages built the same way.
 
 Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
 the host cores instead, on a bounded sample of the same workload.
@@ -163,13 +173,17 @@ class Workload:
         return k.to(self.device), v.to(self.device)
 
     def run_prefill(self, cache):
-        for i, (ls, st) in enumerate(self.prefill):
-            ts, tp = synth.append_positions(ls, st)
-            for c0 in range(0, len(ts), 1 << 20):
-                c1 = min(len(ts), c0 + (1 << 20))
-                k, v = self._rows(c1 - c0, 10_000 + i * 4096 + c0 // (1 << 20))
-                cache.append(k, v, ts[c0:c1].to(self.device), tp[c0:c1].to(self.device), self.page_table)
-                del k, v
+        """Append the untimed prefill; its K/V rows are drawn once and kept for later caches."""
+        if not hasattr(self, "_prefill_rows"):
+            self._prefill_rows = []
+            for i, (ls, st) in enumerate(self.prefill):
+                ts, tp = synth.append_positions(ls, st)
+                for c0 in range(0, len(ts), 1 << 20):
+                    c1 = min(len(ts), c0 + (1 << 20))
+                    k, v = self._rows(c1 - c0, 10_000 + i * 4096 + c0 // (1 << 20))
+                    self._prefill_rows.append((k, v, ts[c0:c1].to(self.device), tp[c0:c1].to(self.device)))
+        for k, v, ts, tp in self._prefill_rows:
+            cache.append(k, v, ts, tp, self.page_table)
 
     def append_bytes(self, mode):
         # read K and V rows (2 x 256 B per head); write bf16 rows (2 x 256 B) or INT4 codes + scale/zero (2 x 68 B)
@@ -235,22 +249,24 @@ def make_cache(w: Workload, mode, b, rv, device, rope=None, code_bits=4):
 
 
 def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False, rope=None, code_bits=4):
-    """Device-timed steps (CUDA events on the launching stream); per-kernel and per-step means (ms).
-    rope: optional (cos, sin) table for the fused rotary embedding; code_bits: 4 or 2."""
+    """Exactly `steps` device-timed steps after `warmup` untimed ones.  Each step is bracketed by
+    CUDA events on the launching stream, with one more between its appends and its decode, so the
+    per-kernel and per-step means (ms) all come from the same timed steps.  L2 is flushed (a
+    256 MiB write) before every step, outside its events.  rope: optional (cos, sin) table for
+    the fused rotary embedding; code_bits: 4 or 2."""
     cache = make_cache(w, mode, b, rv, device, rope, code_bits)
     ws, _ = cache.workspace(w.dec_B, w.max_len, device)
     out = torch.empty(w.dec_B, w.Hq, 128, dtype=torch.bfloat16, device=device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
-    n_split = min(steps, 300)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(max(steps, n_split))]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
 
-    def step(e=None, split=False):
+    def step(e=None):
         if e: e[0].record(stream)
         for k, v, ts, tp in w.appends:
             kvq.kv_append_quant(cache.handle, k, v, k.shape[0], ts, tp, w.page_table, w.pt_stride, w.num_seqs,
                                 stream)
-        if e and split: e[1].record(stream)
+        if e: e[1].record(stream)
         kvq.kv_decode_attn(cache.handle, w.q, w.seq_lens, w.dec_pt, w.pt_stride, w.dec_B, w.max_len, out, 0, ws,
                            ws.numel(), stream)
         if e: e[2].record(stream)
@@ -269,8 +285,6 @@ def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False, r
     _barrier()
     torch.cuda.synchronize(device)
     t0 = time.perf_counter()
-    # whole steps: events at the step boundaries only, so the step's kernels run back to back
-    # (each may start while the one before it finishes: programmatic dependent launch)
     for i in range(steps):
         flush.zero_()  # write 256 MiB > 126 MB L2 between timed steps
         step(evs[i])
@@ -279,14 +293,9 @@ def run_variant(w: Workload, mode, b, rv, steps, warmup, device, clocks=False, r
     _barrier()
     if sampler:
         sampler.__exit__()
-    stp = np.array([e[0].elapsed_time(e[2]) for e in evs[:steps]])
-    # per-kernel times: an event between the append and the decode (they then run in turn)
-    for i in range(n_split):
-        flush.zero_()
-        step(evs[i], split=True)
-    torch.cuda.synchronize(device)
-    app = np.array([e[0].elapsed_time(e[1]) for e in evs[:n_split]])
-    dec = np.array([e[1].elapsed_time(e[2]) for e in evs[:n_split]])
+    stp = np.array([e[0].elapsed_time(e[2]) for e in evs])
+    app = np.array([e[0].elapsed_time(e[1]) for e in evs])
+    dec = np.array([e[1].elapsed_time(e[2]) for e in evs])
     status = cache.get_error()
     cache.close()
     return {"append_ms": float(app.mean()), "decode_ms": float(dec.mean()), "step_ms": float(stp.mean()),
@@ -572,15 +581,121 @@ def reduce_over_ranks(x: float, op: str, device) -> float:
 
 # --------------------------------------------------------------------------- main
 
+# the comparators of every sub-record: naive INT4 and BF16 pages, built the same way
+COMPARATORS = [("int4", kvq.KV_INT4, 0, False), ("bf16", kvq.KV_BF16, 0, False)]
+CONFIG_STEPS = 50  # timed steps of each sub-record variant (after 3 warm-ups)
+
+
+def _dec_kernel(w: Workload, mode):
+    if mode == kvq.KV_BF16:
+        return "bf16_split_kernel + merge_kernel"
+    # the INT4 decode runs the tokens-on-M tile for up to 4 query heads per KV head, else heads-on-M
+    return ("decode_tok_kernel" if w.Hq // w.H <= 4 else "decode_mma_kernel") + " + merge_kernel"
+
+
+def roofline_record(kernel, achieved, peak, peak_kind, traffic=None, **extra):
+    return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+            "traffic": traffic, **extra}
+
+
+def variant_record(w: Workload, mode, r, workload_name, peak, peak_kind, with_traffic=False):
+    """Append and decode rates of one variant's timed steps, each against the HBM roofline."""
+    app_b, dec_b = w.append_bytes(mode), w.decode_bytes(mode)
+    app_gbs = app_b / (r["append_ms"] / 1e3) / 1e9
+    dec_gbs = dec_b / (r["decode_ms"] / 1e3) / 1e9
+    napp = len(w.appends)
+    app_traffic = profiled_traffic("append_kernel", workload_name) if with_traffic else None
+    dkern = _dec_kernel(w, mode)
+    dec_traffic = (profiled_traffic(dkern.split()[0], workload_name)
+                   if with_traffic and mode != kvq.KV_BF16 else None)
+    return {
+        "append": {"us": r["append_ms"] * 1e3, "launches_per_step": napp,
+                   "tokens_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
+                   "algorithmic_bytes": app_b, "algorithmic_bytes_per_launch": app_b / napp, "gbs": app_gbs,
+                   "frac_of_8tbs": app_gbs / NOMINAL_HBM_GBS,
+                   "roofline": roofline_record("append_kernel", app_gbs, peak, peak_kind, app_traffic,
+                                               traffic_unit="DRAM bytes per launch (ncu)")},
+        "decode": {"us": r["decode_ms"] * 1e3, "launches_per_step": 2, "algorithmic_bytes": dec_b, "gbs": dec_gbs,
+                   "frac_of_8tbs": dec_gbs / NOMINAL_HBM_GBS,
+                   "roofline": roofline_record(dkern, dec_gbs, peak, peak_kind, dec_traffic,
+                                               traffic_unit="DRAM bytes of the split kernel per launch (ncu)")},
+        "step_us": r["step_ms"] * 1e3, "steps": r.get("steps"),
+    }
+
+
+def measure_config(name, seed, device, peak, peak_kind, head=None, extend=True, accuracy=True):
+    """Sub-record of one workload: the headline variant, naive INT4 and BF16 pages (batch16: every
+    block size, K and K+V, fused RoPE and 2-bit codes too), the ratios the targets are stated in,
+    and the extend attention where the workload has prefill queries.  head: the headline variant's
+    measurement when it was already taken (the headline workload)."""
+    w = Workload(name, seed, device)
+    hname, hmode, hb, hrv = HEADLINE[name]
+    variants = [(hname, hmode, hb, hrv)] + COMPARATORS
+    if name == "batch16":
+        variants = [(hname, hmode, hb, hrv)] + [v for v in VARIANTS if v[0] != hname]
+    rec = {"description": w.wl.description, "headline_variant": hname, "tokens_appended_per_step": w.tokens_per_step,
+           "append_launches_per_step": len(w.appends), "sequences_decoded_per_step": w.dec_B,
+           "cached_tokens_decoded_per_step": sum(w.dec_lens), "num_q_heads": w.Hq, "page_size": w.ps,
+           "variants": {}}
+    for vname, mode, b, rv in variants:
+        if head is not None and vname == hname:
+            r = head
+        else:
+            r = run_variant(w, mode, b, rv, CONFIG_STEPS, 3, device)
+            r["steps"] = CONFIG_STEPS
+        rec["variants"][vname] = variant_record(w, mode, r, name, peak, peak_kind, with_traffic=(vname == hname))
+    V = rec["variants"]
+    rec["ratios"] = {
+        f"{hname}_over_int4_append_tokens_per_s": V[hname]["append"]["tokens_per_s"] / V["int4"]["append"]["tokens_per_s"],
+        f"{hname}_over_int4_decode_time": V["int4"]["decode"]["us"] / V[hname]["decode"]["us"],
+        "bf16_over_int4_decode_time": V["bf16"]["decode"]["us"] / V["int4"]["decode"]["us"],
+        "bf16_over_int4_step_time": V["bf16"]["step_us"] / V["int4"]["step_us"],
+        f"bf16_over_{hname}_step_time": V["bf16"]["step_us"] / V[hname]["step_us"],
+        "note": "time ratios > 1 mean the second variant is faster; targets: INT4+BDR-128 append and decode "
+                ">= 0.70 of the HBM roofline each, BDR-128 append >= 0.95 of naive INT4"}
+    if name == "batch16":
+        n = CONFIG_STEPS
+        tab = synth.rope_table(max(w.dec_lens) + 1).to(device)
+        r = run_variant(w, kvq.KV_INT4_BDR, 128, False, n, 3, device, rope=tab)
+        rec["bdr128_k_rope"] = {"append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3,
+                                "append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
+                                "note": "fused rotary embedding; plus the table reads (512 B per appended token)"}
+        r = run_variant(w, kvq.KV_INT4_BDR, 128, False, n, 3, device, code_bits=2)
+        rec["bdr128_k_int2"] = {"append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3,
+                                "append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
+                                "note": "2-bit codes; timed like the others, bytes not comparable"}
+        if accuracy:
+            rec["accuracy"] = {"vs": "exact float64 attention on the unquantised bf16 K/V",
+                               "metric": "per (sequence, query head) row max|o-r|/max|r|", **accuracy_study(w, device)}
+    if extend and extend_setup(w) is not None:
+        rec["extend"] = {"what": "kv_extend_attn: causal attention of the step's prefill queries over the paged "
+                                 "cache (one launch), outside the timed step", **run_extend(w, hmode, hb, hrv, 10, device)}
+    del w
+    torch.cuda.empty_cache()
+    return rec
+
+
+def config_dict(w: Workload, variant: str, world: int, seed: int):
+    """The workload the line is quoted on (identical in the kernel and the reference arm)."""
+    return {"workload": w.name, "description": w.wl.description, "variant": variant,
+            "sequences": len(w.lengths), "tokens_appended_per_step": w.tokens_per_step,
+            "append_launches_per_step": len(w.appends), "sequences_decoded_per_step": w.dec_B,
+            "cached_tokens_decoded_per_step": sum(w.dec_lens), "num_kv_heads": w.H, "num_q_heads": w.Hq,
+            "head_dim": 128, "page_size": w.ps, "l2": "256 MiB buffer written before every timed step (L2 is 126 MB)",
+            "parallelism": f"{world} independent replica(s), one per GPU, no collective on the data path",
+            "seed": seed}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
-    ap.add_argument("--workload", default="batch16", choices=list(synth.WORKLOADS))
+    ap.add_argument("--workload", default="mixed256", choices=list(synth.WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload sub-records")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-accuracy", action="store_true")
     ap.add_argument("--no-extend", action="store_true")
@@ -600,102 +715,56 @@ def main():
     device = torch.device("cuda", local)
     w = Workload(args.workload, args.seed + rank, device)  # each rank: its own independent batch
     hname, hmode, hb, hrv = HEADLINE[args.workload]
+    peak, peak_kind = peak_hbm()
 
     res = run_variant(w, hmode, hb, hrv, args.steps, args.warmup, device, clocks=True)
+    res["steps"] = args.steps
     step_ms = reduce_over_ranks(res["step_ms"], "max", device)
+    app_ms = reduce_over_ranks(res["append_ms"], "max", device)
+    dec_ms = reduce_over_ranks(res["decode_ms"], "max", device)
     tokens = reduce_over_ranks(w.tokens_per_step, "sum", device)
-    value = tokens / (step_ms / 1e3)
+    value = tokens / (app_ms / 1e3)  # appended tokens per second of the append kernel's own time
 
-    sweep = {}
-    if not args.no_sweep and args.workload == "batch16":
-        n = max(50, min(args.steps // 4, 500))
-        for name, mode, b, rv in VARIANTS:
-            r = res if name == hname else run_variant(w, mode, b, rv, n, 3, device)
-            sweep[name] = {"append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
-                           "append_gbs": w.append_bytes(mode) / (r["append_ms"] / 1e3) / 1e9,
-                           "decode_gbs": w.decode_bytes(mode) / (r["decode_ms"] / 1e3) / 1e9,
-                           "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3}
-        sweep["bdr128_k_over_int4_append"] = sweep["bdr128_k"]["append_tok_per_s"] / sweep["int4"]["append_tok_per_s"]
-        # the same step with the fused rotary embedding (keys turned in the append, q in the decode)
-        tab = synth.rope_table(max(w.dec_lens) + 1).to(device)
-        r = run_variant(w, kvq.KV_INT4_BDR, 128, False, n, 3, device, rope=tab)
-        sweep["bdr128_k_rope"] = {"append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
-                                  "append_gbs": w.append_bytes(kvq.KV_INT4_BDR) / (r["append_ms"] / 1e3) / 1e9,
-                                  "decode_gbs": w.decode_bytes(kvq.KV_INT4_BDR) / (r["decode_ms"] / 1e3) / 1e9,
-                                  "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3,
-                                  "note": "plus the table reads (512 B per appended token, L2-resident)"}
-        # the 2-bit variant (half the code bytes: 576 B per token-layer instead of 1088)
-        r = run_variant(w, kvq.KV_INT4_BDR, 128, False, n, 3, device, code_bits=2)
-        sweep["bdr128_k_int2"] = {"append_tok_per_s": w.tokens_per_step / (r["append_ms"] / 1e3),
-                                  "append_us": r["append_ms"] * 1e3, "decode_us": r["decode_ms"] * 1e3,
-                                  "note": "2-bit codes; timed like the others, bytes not comparable"}
-
-    extend = None
-    if not args.no_extend and extend_setup(w) is not None:
-        extend = run_extend(w, hmode, hb, hrv, 10, device)
-
-    accuracy = None
-    if not args.no_accuracy and args.workload in ("batch16", "single256"):
-        accuracy = accuracy_study(w, device)
-
-    e2e_ms, h2d, d2h = run_e2e(w, hmode, hb, hrv, max(20, min(200, args.steps // 20)), args.warmup, device)
+    e2e_ms, h2d, d2h = run_e2e(w, hmode, hb, hrv, max(20, min(200, args.steps)), args.warmup, device)
     e2e_ms = reduce_over_ranks(e2e_ms, "max", device)
 
-    peak, peak_kind = peak_hbm()
-    app_b, dec_b = w.append_bytes(hmode), w.decode_bytes(hmode)
-    app_gbs = app_b / (res["append_ms"] / 1e3) / 1e9
-    dec_gbs = dec_b / (res["decode_ms"] / 1e3) / 1e9
+    head = variant_record(w, hmode, res, args.workload, peak, peak_kind, with_traffic=True)
     dominant = "append" if res["append_ms"] >= res["decode_ms"] else "decode"
-    dom_gbs = app_gbs if dominant == "append" else dec_gbs
-    # the INT4 decode runs the tokens-on-M tile for up to 4 query heads per KV head, else heads-on-M
-    dec_kernel = "decode_tok_kernel" if w.Hq // w.H <= 4 else "decode_mma_kernel"
-    dom_kernel = "append_kernel" if dominant == "append" else dec_kernel
-    traffic = profiled_traffic(dom_kernel, args.workload)
-
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32",
         "dtype_detail": "bf16 rows in; fp32 rotation and quantiser; INT4 codes + fp16 scale/zero stored; attention on "
                         "int8 / fp16 tensor-core tiles with int32 / fp32 accumulation", "data": "synthetic",
-        "config": {"workload": args.workload, "description": w.wl.description, "variant": hname,
-                   "sequences": len(w.lengths), "tokens_appended_per_step": w.tokens_per_step,
-                   "sequences_decoded_per_step": w.dec_B, "cached_tokens_decoded_per_step": sum(w.dec_lens),
-                   "num_kv_heads": w.H, "num_q_heads": w.Hq, "head_dim": 128, "page_size": w.ps,
-                   "l2": "256 MiB buffer written between timed steps (L2 is 126 MB)",
-                   "parallelism": f"{world} independent replica(s), one per GPU, no collective on the data path",
-                   "seed": args.seed},
-        "components": {
-            "append": {"us": res["append_ms"] * 1e3, "tokens_per_s": w.tokens_per_step / (res["append_ms"] / 1e3),
-                       "algorithmic_bytes": app_b, "gbs": app_gbs, "frac_of_peak": app_gbs / peak,
-                       "frac_of_8tbs": app_gbs / NOMINAL_HBM_GBS, "launches_per_step": len(w.appends)},
-            "decode": {"us": res["decode_ms"] * 1e3, "algorithmic_bytes": dec_b, "gbs": dec_gbs,
-                       "frac_of_peak": dec_gbs / peak, "frac_of_8tbs": dec_gbs / NOMINAL_HBM_GBS,
-                       "note": "split + merge kernels"}},
-        "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
-                     "frac": dom_gbs / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
-                     "traffic": traffic},
+        "value_detail": "appended tokens per second of the append kernel's own time (CUDA events around the step's "
+                        "appends inside each timed step; all ranks' tokens / the slowest rank's mean append time); "
+                        "ms_per_step is the whole step (appends + decode)",
+        "config": config_dict(w, hname, world, args.seed),
+        "components": {"append": head["append"], "decode": {**head["decode"], "note": "split + merge kernels"}},
+        "decode_gbs": head["decode"]["gbs"], "decode_frac_of_peak": head["decode"]["roofline"]["frac"],
+        "roofline": {**head[dominant]["roofline"], "component": dominant,
+                     "note": "the dominant kernel of the step; both components carry their own roofline"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "what": "the whole step through the C ABI from pinned host buffers: the step's inputs copied to the "
+                        "device and the attention output read back inside the timed region"},
         "gpu_launches": res["launches_per_step"] * args.steps,
         "clocks": res["clocks"],
         "device_status": kvq.status_string(res["status"]),
     }
-    if sweep:
-        line["sweep"] = sweep
-    if extend:
-        line["extend"] = {"what": "kv_extend_attn: causal attention of the step's prefill queries over the "
-                                  "paged cache (one launch), outside the timed step", **extend}
-    if accuracy:
-        line["accuracy"] = {"vs": "exact float64 attention on the unquantised bf16 K/V",
-                            "metric": "per (sequence, query head) row max|o-r|/max|r|", **accuracy}
+    if not args.no_configs:
+        # every workload, each with the headline variant and the comparators built the same way
+        del w
+        torch.cuda.empty_cache()
+        configs = {}
+        for name in synth.WORKLOADS:
+            configs[name] = measure_config(name, args.seed + rank, device, peak, peak_kind,
+                                           head=res if name == args.workload else None,
+                                           extend=not args.no_extend, accuracy=not args.no_accuracy)
+        line["configs"] = configs
+        w = Workload(args.workload, args.seed + rank, device)
     if rank == 0 and world == 1 and not args.no_cpu:
-        # about one step's worth of oracle work per repetition for batch16 (~4 s), bounded for the
-        # large workloads; 3 repetitions: ~10-15 s of host CPU on one core, then the same sample
-        # split over every core
-        Ls = int(min(max(np.mean(w.dec_lens), 16), 32768))
-        nd = max(1, min(w.dec_B, 16, (1 << 20) // (w.Hq * Ls)))
-        kw = dict(tok_budget=min(w.tokens_per_step, 40960), row_budget=w.Hq, dec_seqs=nd, reps=3)
+        kw = cpu_sample(w)
         c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, **kw)
         cores, model = host_cpu()
         line["cpu_baseline"] = {"value": w.tokens_per_step / oracle_step_seconds(w, c_app, c_dec),
@@ -711,33 +780,35 @@ def main():
         _dist.destroy_process_group()
 
 
+def cpu_sample(w: Workload):
+    """The bounded oracle sample of one step of w: up to 40960 appended tokens, and every query head of
+    up to 16 sequences of the workload's mean decoded length (fewer for long sequences, about 1 M
+    (token x query head) units), three repetitions."""
+    Ls = int(min(max(np.mean(w.dec_lens), 16), 32768))
+    nd = max(1, min(w.dec_B, 16, (1 << 20) // (w.Hq * Ls)))
+    return dict(tok_budget=min(w.tokens_per_step, 40960), row_budget=w.Hq, dec_seqs=nd, reps=3)
+
+
 def run_reference(args, world):
-    """The CPU oracle as the reference arm (rank 0 only): each step runs a bounded sample of the
-    workload's step on all the host's cores (its tokens and rows split over threads) and scales
-    its unit costs to the full step."""
+    """The CPU oracle as the reference arm (rank 0 only): each step runs the same bounded sample of
+    the workload's step as the kernel arm's all-core cpu_baseline (its tokens and rows split over
+    every host core), and scales its unit costs to the full step."""
     w = Workload(args.workload, args.seed, torch.device("cpu"))
-    _, hmode, hb, hrv = HEADLINE[args.workload]
-    budget_s = 120.0
+    hname, hmode, hb, hrv = HEADLINE[args.workload]
     cores, model = host_cpu()
-    c_app, c_dec, _ = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=256, row_budget=1)
-    unit = max(oracle_step_seconds(w, c_app, c_dec), 1e-9)
-    frac = min(1.0, budget_s / (args.steps + args.warmup) / unit)
-    tok = max(16, int(min(w.tokens_per_step, 20000) * frac))
-    rows = max(1, int(8 * frac))
+    kw = cpu_sample(w)
     times, sample = [], ""
     for i in range(args.warmup + args.steps):
-        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, tok_budget=tok, row_budget=rows, seed=i,
-                                                 threads=cores)
+        c_app, c_dec, sample = oracle_unit_costs(w, hmode, hb, hrv, seed=i, threads=cores, **kw)
         if i >= args.warmup:
             times.append(oracle_step_seconds(w, c_app, c_dec))
     step_s = float(np.mean(times))
     value = w.tokens_per_step / step_s
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "dtype_detail": "oracle: fp32 write path, float64 attention",
-            "data": "synthetic",
-            "config": {"workload": args.workload, "variant": HEADLINE[args.workload][0],
-                       "sequences": len(w.lengths), "tokens_appended_per_step": w.tokens_per_step},
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "dtype_detail": "oracle: fp32 write path, float64 attention", "data": "synthetic",
+            "config": config_dict(w, hname, world, args.seed),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
                              "cpu_model": model},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -68,3 +68,40 @@ def test_oracle_unit_costs_threads_and_host_cpu():
         assert c_app > 0 and c_dec > 0 and f"{threads} thread(s)" in sample
     cores, model = bench.host_cpu()
     assert cores >= 1 and isinstance(model, str) and model
+
+
+def test_variant_record_rates_and_fractions():
+    """A sub-record's rates are its algorithmic bytes over the measured times, its fractions
+    those rates over the peak, per component."""
+    w = bench.Workload("batch16", 0, torch.device("cpu"))
+    r = {"append_ms": 0.05, "decode_ms": 0.025, "step_ms": 0.08}
+    rec = bench.variant_record(w, kvq.KV_INT4_BDR, r, "batch16", 6544.0, "measured")
+    app_b = w.tokens_per_step * 8 * (2 * 256 + 2 * 68)
+    assert rec["append"]["algorithmic_bytes"] == app_b
+    assert abs(rec["append"]["gbs"] - app_b / 0.05e-3 / 1e9) < 1e-6
+    assert abs(rec["append"]["roofline"]["frac"] - rec["append"]["gbs"] / 6544.0) < 1e-12
+    assert abs(rec["append"]["tokens_per_s"] - w.tokens_per_step / 0.05e-3) < 1e-3
+    dec_b = w.decode_bytes(kvq.KV_INT4_BDR)
+    assert sum(w.dec_lens) * 8 * 136 < dec_b < sum(w.dec_lens) * 8 * 136 * 1.01
+    assert abs(rec["decode"]["roofline"]["frac"] - dec_b / 0.025e-3 / 1e9 / 6544.0) < 1e-12
+    assert rec["decode"]["roofline"]["kernel"].startswith("decode_tok_kernel")
+    w8 = bench.Workload("mixed256", 0, torch.device("cpu"))
+    assert bench._dec_kernel(w8, kvq.KV_INT4_BDR).startswith("decode_mma_kernel")
+
+
+def test_reference_arm_prints_the_kernel_arms_config(capsys):
+    """The reference arm quotes the same workload, variant, metric and unit as the kernel arm, and
+    its sample has the shape of the kernel arm's all-core baseline."""
+    import argparse
+    import json
+
+    args = argparse.Namespace(workload="single256", seed=0, steps=1, warmup=1)
+    bench.run_reference(args, 1)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    w = bench.Workload("single256", 0, torch.device("cpu"))
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "tokens/s"
+    assert line["config"] == bench.config_dict(w, bench.HEADLINE["single256"][0], 1, 0)
+    kw = bench.cpu_sample(w)
+    assert kw["row_budget"] == w.Hq and kw["reps"] >= 3
+    assert f"decode of {w.Hq} query-head rows" in line["cpu_baseline"]["sample"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
