@@ -1,6 +1,6 @@
-// kvq_decode.cu -- paged GQA decode attention: planning, the CUDA-core split
-// kernel used for BF16 pages and the split-K merge kernel.  The INT4 split
-// kernel (tensor cores) is in kvq_decode_mma.cu.
+// kvq_decode.cu -- paged GQA decode attention: planning and the split-K merge
+// kernel.  The split kernels (tensor cores) are in kvq_decode_mma.cu (INT4 pages)
+// and kvq_decode_bf16.cu (BF16 pages).
 //
 // SAW-INT4 (wispaper.ai blog, section 3): the query is rotated in step with
 // H_blk at inference, so (q H)(k H)^T = q k^T and attention runs directly on
@@ -24,9 +24,6 @@ constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
 using Params = DecodeParams;
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -36,189 +33,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
-}
-
-// ---------------------------------------------------- CUDA-core split (BF16) ---
-
-// One CTA per (split k, KV head h, sequence s) over bf16 pages.  Lanes own tokens
-// for q.k and head_dim slices for P.V (staged per warp), online softmax per query
-// head, the 4 warps merged in shared memory.
-template <int G>
-struct Bf16Smem {
-    float qs[G][kHeadDim];
-    union {
-        struct {
-            float pt[kWarps][32][G];
-            uint32_t v[kWarps][32][65];  // staged V rows (+1 word: no bank conflicts)
-        } loop;
-        struct {
-            float m[kWarps][G];
-            float l[kWarps][G];
-            float o[kWarps][G][kHeadDim];
-        } merge;
-    } u;
-};
-
-template <int G>
-__global__ void __launch_bounds__(kThreads) bf16_split_kernel(Params p) {
-    __shared__ Bf16Smem<G> sm;
-    const int k = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = p.g.H, Hq = p.g.Hq, ps = p.g.page_size;
-    const int L = decode_len(p, s);
-    if (k == 0 && h == 0 && tid == 0 && L != __ldg(p.a.seq_lens + s)) flag_error(p.err, kErrOOB);
-    const int t0 = k * p.item_tokens;
-    if (t0 >= L) {  // past the end of the sequence
-        grid_dep_wait();  // still: no grid here completes before the one it follows
-        grid_dep_launch();
-        return;
-    }
-    const int t1 = min(L, t0 + p.item_tokens);
-    const int64_t out_row0 = partial_row(p, s, k, h * G);
-
-    const uint16_t* q = static_cast<const uint16_t*>(p.a.q) + (int64_t(s) * Hq + h * G) * kHeadDim;
-    if (p.g.rope) {  // fused rotary embedding at position seq_len - 1: pairs (i, i + 64)
-#pragma unroll
-        for (int g = 0; g < G; ++g) sm.qs[g][tid] = __uint_as_float(uint32_t(q[g * kHeadDim + tid]) << 16);
-        __syncthreads();
-        const int pos = __ldg(p.a.seq_lens + s) - 1;
-        const int i = tid & 63;
-        const float c = __ldg(p.g.rope + int64_t(pos) * kHeadDim + 2 * i);
-        const float sn = __ldg(p.g.rope + int64_t(pos) * kHeadDim + 2 * i + 1);
-        float turned[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float own = sm.qs[g][tid], other = sm.qs[g][tid ^ 64];
-            turned[g] = tid < 64 ? fmaf(own, c, -other * sn) : fmaf(own, c, other * sn);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int g = 0; g < G; ++g) sm.qs[g][tid] = turned[g] * p.qscale;
-    } else {
-#pragma unroll
-        for (int g = 0; g < G; ++g) sm.qs[g][tid] = __uint_as_float(uint32_t(q[g * kHeadDim + tid]) << 16) * p.qscale;
-    }
-    __syncthreads();
-
-    float m[G], lsum[G], o[G][4];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m[g] = -INFINITY;
-        lsum[g] = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[g][e] = 0.0f;
-    }
-    const int32_t* pt = p.a.page_table + int64_t(s) * p.a.pt_stride;
-    grid_dep_wait();  // the cache as the previous grid (an append) left it
-    grid_dep_launch();
-
-    for (int base = t0 + 32 * warp; base < t1; base += 32 * kWarps) {
-        const int t = base + lane;
-        bool valid = t < t1;
-        int64_t row = 0;
-        if (valid) {
-            const int page = __ldg(pt + page_of_pos(p, t));
-            if (page < 0 || page >= p.g.num_pages) {
-                flag_error(p.err, kErrOOB);
-                valid = false;
-            } else {
-                row = (int64_t(page) * H + h) * ps + slot_of_pos(p, t);
-            }
-        }
-        float sc[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) sc[g] = -INFINITY;
-        if (valid) {
-            float acc[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g) acc[g] = 0.0f;
-            const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.g.k_pool) + row * 256);
-#pragma unroll 4
-            for (int j = 0; j < 16; ++j) {
-                const uint4 w = __ldg(kr + j);
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float k0 = bf16_lo(ww[e]), k1 = bf16_hi(ww[e]);
-                    const int d = 8 * j + 2 * e;
-#pragma unroll
-                    for (int g = 0; g < G; ++g) acc[g] += sm.qs[g][d] * k0 + sm.qs[g][d + 1] * k1;
-                }
-            }
-#pragma unroll
-            for (int g = 0; g < G; ++g) sc[g] = acc[g];
-        }
-        float pg[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float mnew = fmaxf(m[g], warp_max(sc[g]));
-            const float alpha = (mnew == -INFINITY) ? 1.0f : exp2f(m[g] - mnew);
-            pg[g] = valid ? exp2f(sc[g] - mnew) : 0.0f;
-            m[g] = mnew;
-            lsum[g] = lsum[g] * alpha + pg[g];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[g][e] *= alpha;
-        }
-        uint32_t* vs = sm.u.loop.v[warp][lane];
-        if (valid) {
-            const uint4* vr = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.g.v_pool) + row * 256);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const uint4 w = __ldg(vr + j);
-                vs[4 * j + 0] = w.x;
-                vs[4 * j + 1] = w.y;
-                vs[4 * j + 2] = w.z;
-                vs[4 * j + 3] = w.w;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 64; ++j) vs[j] = 0u;
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g) sm.u.loop.pt[warp][lane][g] = pg[g];
-        __syncwarp();
-        const int ntok = min(32, t1 - base);
-        for (int j = 0; j < ntok; ++j) {
-            const uint32_t w0 = sm.u.loop.v[warp][j][2 * lane], w1 = sm.u.loop.v[warp][j][2 * lane + 1];
-            const float vv[4] = {bf16_lo(w0), bf16_hi(w0), bf16_lo(w1), bf16_hi(w1)};
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float wgt = sm.u.loop.pt[warp][j][g];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[g][e] += wgt * vv[e];
-            }
-        }
-        __syncwarp();
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) lsum[g] = warp_sum(lsum[g]);
-    __syncthreads();
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        if (lane == 0) {
-            sm.u.merge.m[warp][g] = m[g];
-            sm.u.merge.l[warp][g] = lsum[g];
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sm.u.merge.o[warp][g][4 * lane + e] = o[g][e];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm.u.merge.m[w][g]);
-        float acc = 0.0f, lt = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float mw = sm.u.merge.m[w][g];
-            const float f = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
-            acc += f * sm.u.merge.o[w][g][tid];
-            lt += f * sm.u.merge.l[w][g];
-        }
-        p.ws_o[(out_row0 + g) * kHeadDim + tid] = acc;
-        if (tid == 0) p.ws_ml[out_row0 + g] = make_float2(M, lt);
-    }
 }
 
 // ---------------------------------------------------------------- merge --------
@@ -294,15 +108,9 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(Params p, int rotate_ou
 
 template <int G>
 cudaError_t launch_group(const Params& p, cudaStream_t st) {
-    const int B = p.a.batch, H = p.g.H;
-    cudaError_t e;
-    if (p.g.mode == 0) {
-        e = launch_overlapped(bf16_split_kernel<G>, dim3(p.max_splits, H, B), dim3(kThreads), 0, st, p);
-    } else {
-        e = launch_decode_mma(p, st);
-    }
+    const cudaError_t e = p.g.mode == 0 ? launch_decode_bf16(p, st) : launch_decode_mma(p, st);
     if (e != cudaSuccess) return e;
-    return launch_overlapped(merge_kernel, dim3(B * p.g.Hq), dim3(kThreads), 0, st, p,
+    return launch_overlapped(merge_kernel, dim3(p.a.batch * p.g.Hq), dim3(kThreads), 0, st, p,
                              int(p.g.mode == 2 && p.g.rotate_v));
 }
 

@@ -74,5 +74,7 @@ __device__ __forceinline__ float fast_exp2(float x) {  // MUFU ex2; exp2(-inf) =
 
 // Tensor-core split kernel for the INT4 modes (grid: max_splits x H x B).
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s);
+// Tensor-core split kernel for BF16 pages (grid: max_splits x H x B).
+cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t s);
 
 }  // namespace kvq

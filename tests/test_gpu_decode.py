@@ -64,12 +64,41 @@ def test_decode_group_sizes(G):
     _run(c, lengths)
 
 
-def test_decode_long_sequence_many_splits():
+@pytest.mark.parametrize("mode,b", [(kvq.KV_INT4_BDR, 128), (kvq.KV_BF16, 0)], ids=["bdr128k", "bf16"])
+def test_decode_long_sequence_many_splits(mode, b):
     """One 40k-token sequence, page size 64: split-K across the context, then the merge."""
     wl = synth.Workload("t", 8, 32, 128, 64, synth.OUTLIERS_1PCT, "test")
     lengths = [40_000]
-    c = make_case(kvq.KV_INT4_BDR, 128, False, lengths, wl, seed=2)
+    c = make_case(mode, b, False, lengths, wl, seed=2)
     _run(c, lengths)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_decode_bf16_group_sizes_nan_filled_pool(G):
+    """BF16 pages, every group size.  The pools hold NaN bits before the append, so the slots
+    past each sequence's end, which its last 16-token chunk copies too, are NaN; a page id
+    outside the pool is skipped.  Masked rows must never reach the P.V product."""
+    wl = synth.Workload("t", 4, 4 * G, 128, 16, synth.OUTLIERS_X20, "test")
+    lengths = [1, 17, 333, 2100]
+    c = make_case(kvq.KV_BF16, 0, False, lengths, wl, seed=10 + G)
+    for t in (c.cache.k_pool, c.cache.v_pool):
+        t.view(torch.uint8).fill_(0xFF)
+    assert gpu_append(c) == kvq.KV_OK
+    oracle_append(c)
+    q = synth.make_q(len(lengths), 4 * G, 128, seed=3)
+    ref, _ = oracle_decode(c, q, lengths)
+    out, st = gpu_decode(c, q, lengths)
+    assert st == kvq.KV_OK
+    assert torch.isfinite(out).all()
+    assert attn_rel_err(out.cpu().numpy(), ref) <= ATTN_RTOL
+    pt = c.page_table.clone()
+    pt[3, 5] = -7
+    out, st = gpu_decode(c, q, lengths, page_table=pt)
+    assert st == kvq.KV_ERR_OOB
+    ref, skipped = oracle_decode(c, q, lengths, page_table=pt)
+    assert skipped == 16 * 4 * G
+    assert torch.isfinite(out).all()
+    assert attn_rel_err(out.cpu().numpy(), ref) <= ATTN_RTOL
 
 
 def test_decode_empty_and_loose_bound():
