@@ -10,9 +10,11 @@
 // quantiser and the packing then run in registers with no shuffles; the fp32
 // butterflies use sm_100's packed f32x2 adds, pairing element i with element
 // i + 64 so every stage of stride < 64 is one packed op per pair.  The compiler
-// contracts a packed multiply followed by a packed add into one fused op even
-// when both carry an explicit rounding mode, so the only packed multiply used
-// is a deliberate fma, and the 1/sqrt(b) normalisation is scalar.
+// contracts the packed multiply intrinsic followed by a packed add into one fused
+// op even when both carry an explicit rounding mode, so the 1/sqrt(b)
+// normalisation is a packed multiply written in PTX, which it leaves alone.  K
+// and V rows that take the same path (no rotation, or both rotated) share one
+// instantiation of it: half the hot code, fewer instruction-fetch stalls.
 //
 // Data movement: a persistent grid (one CTA per SM); per CTA a ring of three
 // 56 KiB shared-memory stages filled by TMA tensor loads (128-byte swizzle,
@@ -116,10 +118,19 @@ __device__ __forceinline__ void load_row(const uint8_t* stage, int row, float2 (
     }
 }
 
+// fp32x2 multiply as packed PTX: the compiler keeps it a separate rounding from the adds
+// that follow (it contracts the packed multiply intrinsic with a following packed add)
+__device__ __forceinline__ float2 f2_mul_rn(float2 a, float s) {
+    unsigned long long v = (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+    const unsigned long long m = (static_cast<unsigned long long>(__float_as_uint(s)) << 32) | __float_as_uint(s);
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(v) : "l"(v), "l"(m));
+    return make_float2(__uint_as_float(uint32_t(v)), __uint_as_float(uint32_t(v >> 32)));
+}
+
 // Block-diagonal normalised Sylvester-Hadamard rotation of one row, fp32,
 // stages of increasing stride, then the 1/sqrt(b) multiply.  The butterflies
 // are packed adds (no multiply anywhere to contract with); the normalisation
-// uses scalar multiplies that are never merged into a later add.
+// is a packed multiply in PTX that is never merged into a later add.
 template <int BLK>
 __device__ __forceinline__ void rotate_row(float2 (&R)[64], float r_b) {
     constexpr int kPacked = BLK < 64 ? BLK : 64;  // strides below 64 stay within a packed lane
@@ -139,7 +150,7 @@ __device__ __forceinline__ void rotate_row(float2 (&R)[64], float r_b) {
         for (int i = 0; i < 64; ++i) R[i] = make_float2(__fadd_rn(R[i].x, R[i].y), __fsub_rn(R[i].x, R[i].y));
     }
 #pragma unroll
-    for (int i = 0; i < 64; ++i) R[i] = make_float2(__fmul_rn(R[i].x, r_b), __fmul_rn(R[i].y, r_b));
+    for (int i = 0; i < 64; ++i) R[i] = f2_mul_rn(R[i], r_b);
 }
 
 // Codes of a row into 16 packed words: wa = elements 0..63, wb = elements 64..127.
@@ -478,6 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int seqno = 0, n = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++n) {
         int2 m = make_int2(-1, 0);
+#pragma unroll 1
         for (int kv = 0; kv < 2; ++kv, ++seqno) {
             const int e = seqno % kStages;
             const uint32_t fill = seqno / kStages;
@@ -504,10 +516,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                     uint8_t* cdst = static_cast<uint8_t*>(kv ? p.g.v_pool : p.g.k_pool) + row * (16 * CB);
                     uint32_t* sdst = (kv ? p.g.v_sz : p.g.k_sz) + row;
-                    if (kv == 0)
+                    if (MODE != 2 || ROTV)  // K and V rows take the same path: one copy of it
                         process_row<MODE == 2, BLK, CB>(stage, tid, p.r_b, ROPE ? cs : nullptr, cdst, sdst);
+                    else if (kv == 0)
+                        process_row<true, BLK, CB>(stage, tid, p.r_b, ROPE ? cs : nullptr, cdst, sdst);
                     else
-                        process_row<MODE == 2 && ROTV, BLK, CB>(stage, tid, p.r_b, nullptr, cdst, sdst);
+                        process_row<false, BLK, CB>(stage, tid, p.r_b, nullptr, cdst, sdst);
                 }
             }
             __syncwarp();
