@@ -1,6 +1,7 @@
-// kvq_extend.cu -- extend (chunked-prefill) attention over the paged INT4 cache on the
-// tensor cores: the queries of a sequence's newest tokens, whose keys and values the
-// append has already written, attend causally to the cached tokens.
+// kvq_extend.cu -- extend (chunked-prefill) attention over the paged cache with 2-bit codes
+// on the mma.sync tensor cores (4-bit codes take the tcgen05 kernel in kvq_extend_tc.cu):
+// the queries of a sequence's newest tokens, whose keys and values the append has already
+// written, attend causally to the cached tokens.
 //
 // SAW-INT4's abstract keeps fused attention over the paged quantised layout as a
 // serving constraint; chunked prefill in mixed serving reads the cache this way.  Query
@@ -448,6 +449,8 @@ cudaError_t launch_extend(const CacheGeom& g, const ExtendArgs& a, int* err_word
     ep.d.err = err_word;
     ep.q_indptr = a.q_indptr;
     ep.max_q_len = a.max_q_len;
+    // 4-bit codes: the tcgen05 kernel (kvq_extend_tc.cu); 2-bit codes: the mma.sync kernel below
+    if (g.code_bits == 4) return launch_extend_tc(ep.d, a.q_indptr, a.max_q_len, s);
     const int qb = extend_queries_per_cta(g);
     const dim3 grid((a.max_q_len + qb - 1) / qb, g.H, a.batch);
     switch (g.Hq / g.H) {
