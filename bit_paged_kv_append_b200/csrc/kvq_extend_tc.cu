@@ -65,6 +65,7 @@ struct TcSmem {
     float2 ksz[kTcBlock];   // (scale, zero) of the block's keys
     float2 vsz[kTcBlock];   // (scale, zero + 8 scale) of its values
     uint32_t vmask;         // tokens of the block on valid pages
+    float vmax[4];          // per warp: the largest value scale of its eight tokens
     int tmax, tmin;         // longest / shortest row of the CTA
     uint64_t bar;           // MMA completion
     uint32_t tmem;          // TMEM base column
@@ -116,6 +117,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&v)[32]) {
           "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
           "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
           "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(addr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 16 consecutive TMEM columns of this warp's 32 lanes
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
         : "r"(addr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -196,7 +207,10 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
     if (rowlen >= 0) atomicMin(&sm.tmin, rowlen);
 
     // ---------------- q' of row r: turned, rotated, scaled, split into fp16 parts ----------------
-    float qsum = 0.0f, qexp = 0.0f;  // sum of q' (for the zero term); 2^(24 - e): S -> q'.c
+    // score of a token = qexp (ksc S + zq kz) in log2 units, S the q.K accumulator, (ksc, kz) the
+    // key's scale and zero: qexp = 2^(24 - e) undoes the code scale and the row's power of two,
+    // zq = sum(q') / qexp carries the zero term
+    float qsum = 0.0f, qexp = 1.0f;
     {
         float x[kHeadDim];
         if (rowlen > 0) {
@@ -287,8 +301,13 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
     grid_dep_wait();
     grid_dep_launch();
 
-    // ---- block loader: thread tid copies quarter qq of token tt of each block ----
-    const int tt = tid >> 2, qq = tid & 3;
+    const float zq = qsum / qexp;
+    const float tau = kTau / qexp;  // the reference threshold in the units of ksc S + zq kz
+
+    // ---- block loader: lane L of warp w copies quarter L >> 3 of token 8 w + (L & 7) of each block
+    // (the eight lanes of a store phase fill the eight rows of one core matrix) ----
+    const int lane = tid & 31;
+    const int tt = 8 * warp + (lane & 7), qq = lane >> 3;
     const int32_t* pt = p.a.page_table + int64_t(s) * p.a.pt_stride;
     const uint8_t* kpool = static_cast<const uint8_t*>(p.g.k_pool);
     const uint8_t* vpool = static_cast<const uint8_t*>(p.g.v_pool);
@@ -316,15 +335,14 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
     };
     fetch(0);
 
-    // ---- per-row softmax state ----
-    float O[kHeadDim];  // folded output (fp32, ordinary rounding), relative to m_ref, unscaled by 2^-k
+    // ---- per-row softmax state: O, l and Z in units of 2^-k, relative to the reference m ----
+    float O[kHeadDim];  // folded output (fp32, ordinary rounding)
 #pragma unroll
     for (int d = 0; d < kHeadDim; ++d) O[d] = 0.0f;
     float m_ref = -INFINITY, l = 0.0f, Zs = 0.0f;
-    int k_ref = 0;         // P = p scale_v 2^-k_ref
-    bool dirty = false;    // TMEM O holds something of this row since the last fold
-    uint32_t acc = 0;      // the next P.V accumulates onto TMEM O (0: restart)
-    int since_fold = 0;
+    int k_ref = 0;       // P = p scale_v 2^-k, k the same for every row of the CTA
+    uint32_t acc = 0;    // the next P.V accumulates onto TMEM O (0: restart)
+    int since_fold = 0;  // blocks accumulated in TMEM O since it was last folded
     uint32_t phase = 0;
     bool ok = true;
     const uint32_t s_addr = tm_row + 0, o_addr = tm_row + kTcOCol;
@@ -335,9 +353,7 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
             const bool tok = nok;
             const uint4 ck = nk, cv = nv;
             const uint32_t cks = nks, cvs = nvs;
-            uint32_t* kt = reinterpret_cast<uint32_t*>(sm.k);
             uint8_t* vt = sm.v[j & 1];
-            // key codes: dims 32 qq .. 32 qq + 31 = 4 chunks of 8 dims of row tt
             const uint32_t kw[4] = {ck.x, ck.y, ck.z, ck.w}, vw[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -348,19 +364,21 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
                 *reinterpret_cast<uint4*>(sm.k + kmaj(tt, d0, kHeadDim)) = make_uint4(ko[0], ko[1], ko[2], ko[3]);
                 *reinterpret_cast<uint4*>(vt + nmaj(tt, d0, kHeadDim)) = make_uint4(vo[0], vo[1], vo[2], vo[3]);
             }
-            (void)kt;
+            float vmx = 0.0f;
             if (qq == 0) {
                 const float ksc = half_lo(cks), kzr = half_hi(cks);
                 const float vsc = half_lo(cvs), vzr = half_hi(cvs);
                 sm.ksz[tt] = tok ? make_float2(ksc, kzr) : make_float2(0.0f, 0.0f);
                 sm.vsz[tt] = tok ? make_float2(vsc, vzr + 8.0f * vsc) : make_float2(0.0f, 0.0f);
+                vmx = tok ? fabsf(vsc) : 0.0f;
             }
-            const uint32_t bal = __ballot_sync(0xffffffffu, tok && qq == 0);  // lanes 4 i: token 8 w + i
-            if ((tid & 31) == 0) {
-                uint32_t m8 = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) m8 |= ((bal >> (4 * i)) & 1u) << i;
-                reinterpret_cast<volatile uint8_t*>(&sm.vmask)[warp] = uint8_t(m8);
+            vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, 1));
+            vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, 2));
+            vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, 4));
+            const uint32_t bal = __ballot_sync(0xffffffffu, tok && qq == 0);  // lane i < 8: token 8 w + i
+            if (lane == 0) {
+                reinterpret_cast<volatile uint8_t*>(&sm.vmask)[warp] = uint8_t(bal & 0xFFu);
+                sm.vmax[warp] = vmx;
             }
         }
         fetch(j + 1);  // in flight while the block is computed
@@ -381,6 +399,15 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
             }
             mma_commit(&sm.bar);
         }
+        // the block's power of two for P (the same for every row): 2^8 * max scale 2^-k < 2^15
+        int k_new = k_ref;
+        {
+            const float vmx = fmaxf(fmaxf(sm.vmax[0], sm.vmax[1]), fmaxf(sm.vmax[2], sm.vmax[3]));
+            if (vmx > 0.0f && vmx < INFINITY) {
+                const int k_target = max(-100, min(100, int((__float_as_uint(vmx) >> 23) & 0xFF) - 127 - 6));
+                k_new = since_fold == 0 ? k_target : max(k_ref, k_target);
+            }
+        }
         if (!tc_wait(&sm.bar, phase)) {
             flag_error(p.err, kErrTimeout);
             sm.abort = 1;
@@ -388,66 +415,52 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
         phase ^= 1;
         tc_after_sync();
         // ---------------- 3. scores and the online softmax of row r ----------------
-        uint32_t Sv[kTcBlock];
-        tmem_ld32(s_addr, Sv);
+        uint32_t sc[kTcBlock];  // S, then ksc S + zq kz (the score / qexp) as float bits, -inf when masked
+        tmem_ld32(s_addr, sc);
         const int tb = j * kTcBlock;
         const uint32_t vmask = sm.vmask;
         const bool full = (tb + kTcBlock <= tmin) && (vmask == 0xFFFFFFFFu);
-        float sc[kTcBlock];
         float mblk = -INFINITY;
 #pragma unroll
         for (int t = 0; t < kTcBlock; ++t) {
             const float2 kz = sm.ksz[t];
-            const float v = fmaf(__uint_as_float(Sv[t]) * qexp, kz.x, kz.y * qsum);
-            const bool live = full ? (rowlen > 0) : ((tb + t < rowlen) && ((vmask >> t) & 1u));
-            sc[t] = live ? v : -INFINITY;
-            mblk = fmaxf(mblk, sc[t]);
+            const float v = fmaf(kz.x, __uint_as_float(sc[t]), zq * kz.y);
+            const float vm = (full || ((tb + t < rowlen) && ((vmask >> t) & 1u))) ? v : -INFINITY;
+            sc[t] = __float_as_uint(vm);
+            mblk = fmaxf(mblk, vm);
         }
-        // where the reference max and the P scale go, and whether TMEM O must be folded first
-        const float m_new = (mblk > m_ref + kTau || (m_ref == -INFINITY && mblk > -INFINITY)) ? mblk : m_ref;
-        float pmax = 0.0f;
-#pragma unroll
-        for (int t = 0; t < kTcBlock; ++t) {
-            const float pr = (sc[t] == -INFINITY) ? 0.0f : fast_exp2(sc[t] - m_new);
-            sc[t] = pr;
-            pmax = fmaxf(pmax, pr * sm.vsz[t].x);
-        }
-        int k_new = k_ref;
-        const float pscaled = pmax * pow2i(-k_ref);
-        if (pscaled >= 16384.0f || (pmax > 0.0f && pscaled < 1.0f / 1024.0f && !dirty))  // pmax 2^-k_new in [2^13, 2^14)
-            k_new = max(-100, min(100, int((__float_as_uint(pmax) >> 23) & 0xFF) - 127 - 13));
-        const bool moves = (m_new != m_ref) || (k_new != k_ref);
-        const bool fold = __syncthreads_or((moves && dirty) || since_fold >= kFoldEvery || sm.abort) != 0;
+        const float m_new = (mblk > m_ref + tau || (m_ref == -INFINITY && mblk > -INFINITY)) ? mblk : m_ref;
+        const bool fold = __syncthreads_or((since_fold > 0 && (m_new != m_ref || k_new != k_ref)) ||
+                                           since_fold >= kFoldEvery || sm.abort) != 0;
         if (sm.abort) {  // a wait gave up: let what was issued finish (bounded) before TMEM is freed
             tc_wait(&sm.bar, phase ^ 1);
             ok = false;
             break;
         }
-        if (fold) {
-            // TMEM O (every P.V so far is complete: the q.K commit waited for above came after it)
-            const float f = pow2i(k_ref);
+        if (fold) {  // every P.V so far is complete: the q.K commit waited for above came after it
 #pragma unroll
-            for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
-                uint32_t ov[32];
-                tmem_ld32(o_addr + c0, ov);
+            for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
+                uint32_t ov[16];
+                tmem_ld16(o_addr + c0, ov);
 #pragma unroll
-                for (int d = 0; d < 32; ++d) O[c0 + d] = fmaf(__uint_as_float(ov[d]), f, O[c0 + d]);
+                for (int d = 0; d < 16; ++d) O[c0 + d] += __uint_as_float(ov[d]);
             }
             acc = 0;
             since_fold = 0;
-            dirty = false;
         }
-        if (m_new != m_ref) {
-            const float alpha = (m_ref == -INFINITY) ? 0.0f : fast_exp2(m_ref - m_new);
+        if (m_new != m_ref || k_new != k_ref) {
+            const float alpha =
+                (m_ref == -INFINITY) ? 0.0f : fast_exp2(qexp * (m_ref - m_new)) * pow2i(k_ref - k_new);
 #pragma unroll
             for (int d = 0; d < kHeadDim; ++d) O[d] *= alpha;
             l *= alpha;
             Zs *= alpha;
             m_ref = m_new;
+            k_ref = k_new;
         }
-        k_ref = k_new;
-        const float kd = pow2i(-k_ref);
-        // P parts of row r: tokens 8 c .. 8 c + 7 per 16-byte chunk
+        // p 2^-k = 2^(qexp (v - m) - k); P = p scale_v 2^-k as fp16 high and low parts, tokens 8 c .. 8 c + 7
+        const float cofs = (m_ref == -INFINITY) ? 0.0f : -qexp * m_ref - float(k_ref);
+        float lb = 0.0f;
 #pragma unroll
         for (int c = 0; c < kTcBlock / 8; ++c) {
             uint32_t hw[4], lw[4];
@@ -455,20 +468,22 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
             for (int e = 0; e < 4; ++e) {
                 const int t0 = 8 * c + 2 * e;
                 const float2 v0 = sm.vsz[t0], v1 = sm.vsz[t0 + 1];
-                const float p0 = sc[t0], p1 = sc[t0 + 1];
-                l += p0 + p1;
+                const float p0 = fast_exp2(fmaf(__uint_as_float(sc[t0]), qexp, cofs));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(sc[t0 + 1]), qexp, cofs));
+                lb += p0 + p1;
                 Zs = fmaf(p0, v0.y, fmaf(p1, v1.y, Zs));
-                const float a = p0 * v0.x * kd, b = p1 * v1.x * kd;
-                const uint32_t ha = h_bits(a), hb = h_bits(b);
-                hw[e] = ha | (hb << 16);
-                lw[e] = h_bits(a - __half2float(__ushort_as_half(uint16_t(ha)))) |
-                        (h_bits(b - __half2float(__ushort_as_half(uint16_t(hb)))) << 16);
-                if (p0 > 0.0f || p1 > 0.0f) dirty = true;
+                const float a = p0 * v0.x, b = p1 * v1.x;
+                const __half2 hi2 = __floats2half2_rn(a, b);
+                const float2 back = __half22float2(hi2);
+                const __half2 lo2 = __floats2half2_rn(a - back.x, b - back.y);
+                hw[e] = *reinterpret_cast<const uint32_t*>(&hi2);
+                lw[e] = *reinterpret_cast<const uint32_t*>(&lo2);
             }
             const uint32_t off = kmaj(tid, 8 * c, kTcBlock);
             *reinterpret_cast<uint4*>(sm.p[0] + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             *reinterpret_cast<uint4*>(sm.p[1] + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
+        l += lb;
         ++since_fold;
         fence_proxy_async();
         tc_before_sync();
@@ -500,13 +515,12 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
         tc_after_sync();
     }
     if (ok && nblocks > 0) {
-        const float f = pow2i(k_ref);
 #pragma unroll
-        for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
-            uint32_t ov[32];
-            tmem_ld32(o_addr + c0, ov);
+        for (int c0 = 0; c0 < kHeadDim; c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld16(o_addr + c0, ov);
 #pragma unroll
-            for (int d = 0; d < 32; ++d) O[c0 + d] = fmaf(__uint_as_float(ov[d]), f, O[c0 + d]);
+            for (int d = 0; d < 16; ++d) O[c0 + d] += __uint_as_float(ov[d]);
         }
     }
     tc_before_sync();
