@@ -314,11 +314,19 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
     uint4 nk = make_uint4(0, 0, 0, 0), nv = make_uint4(0, 0, 0, 0);
     uint32_t nks = 0, nvs = 0;
     bool nok = false;
-    auto fetch = [&](int j) {  // raw codes of block j into the prefetch registers
+    // page id of this thread's token in block j: loaded one block before the codes, so that the
+    // code loads never wait for it
+    auto page_id = [&](int j) -> int {
         const int T = j * kTcBlock + tt;
+        return (j < nblocks && T < tmax) ? __ldg(pt + page_of_pos(p, T)) : -1;
+    };
+    int npage = page_id(0);
+    auto fetch = [&](int j) {  // raw codes of block j into the prefetch registers; then block j + 1's page id
+        const int T = j * kTcBlock + tt;
+        const int page = npage;
+        npage = page_id(j + 1);
         nok = false;
         if (j < nblocks && T < tmax) {
-            const int page = __ldg(pt + page_of_pos(p, T));
             if (page >= 0 && page < p.g.num_pages) {
                 const int64_t row = (int64_t(page) * p.g.H + h) * p.g.page_size + slot_of_pos(p, T);
                 nk = __ldg(reinterpret_cast<const uint4*>(kpool + row * 64) + qq);
@@ -341,6 +349,7 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
     for (int d = 0; d < kHeadDim; ++d) O[d] = 0.0f;
     float m_ref = -INFINITY, l = 0.0f, Zs = 0.0f;
     int k_ref = 0;       // P = p scale_v 2^-k, k the same for every row of the CTA
+    bool k_set = false;
     uint32_t acc = 0;    // the next P.V accumulates onto TMEM O (0: restart)
     int since_fold = 0;  // blocks accumulated in TMEM O since it was last folded
     uint32_t phase = 0;
@@ -399,13 +408,20 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
             }
             mma_commit(&sm.bar);
         }
-        // the block's power of two for P (the same for every row): 2^8 * max scale 2^-k < 2^15
+        // the power of two for P, the same for every row: 2^8 * max scale 2^-k < 2^15.  It is set at
+        // the first block with values, with room for scales 16 times larger, and raised (which needs
+        // a fold) only when a block's values exceed that.
         int k_new = k_ref;
         {
             const float vmx = fmaxf(fmaxf(sm.vmax[0], sm.vmax[1]), fmaxf(sm.vmax[2], sm.vmax[3]));
             if (vmx > 0.0f && vmx < INFINITY) {
                 const int k_target = max(-100, min(100, int((__float_as_uint(vmx) >> 23) & 0xFF) - 127 - 6));
-                k_new = since_fold == 0 ? k_target : max(k_ref, k_target);
+                if (!k_set) {
+                    k_new = min(100, k_target + 4);
+                    k_set = true;
+                } else {
+                    k_new = max(k_ref, k_target);
+                }
             }
         }
         if (!tc_wait(&sm.bar, phase)) {
@@ -420,15 +436,16 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
         const int tb = j * kTcBlock;
         const uint32_t vmask = sm.vmask;
         const bool full = (tb + kTcBlock <= tmin) && (vmask == 0xFFFFFFFFu);
-        float mblk = -INFINITY;
+        float mb4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int t = 0; t < kTcBlock; ++t) {
             const float2 kz = sm.ksz[t];
             const float v = fmaf(kz.x, __uint_as_float(sc[t]), zq * kz.y);
             const float vm = (full || ((tb + t < rowlen) && ((vmask >> t) & 1u))) ? v : -INFINITY;
             sc[t] = __float_as_uint(vm);
-            mblk = fmaxf(mblk, vm);
+            mb4[t & 3] = fmaxf(mb4[t & 3], vm);
         }
+        const float mblk = fmaxf(fmaxf(mb4[0], mb4[1]), fmaxf(mb4[2], mb4[3]));
         const float m_new = (mblk > m_ref + tau || (m_ref == -INFINITY && mblk > -INFINITY)) ? mblk : m_ref;
         const bool fold = __syncthreads_or((since_fold > 0 && (m_new != m_ref || k_new != k_ref)) ||
                                            since_fold >= kFoldEvery || sm.abort) != 0;
@@ -460,7 +477,7 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
         }
         // p 2^-k = 2^(qexp (v - m) - k); P = p scale_v 2^-k as fp16 high and low parts, tokens 8 c .. 8 c + 7
         const float cofs = (m_ref == -INFINITY) ? 0.0f : -qexp * m_ref - float(k_ref);
-        float lb = 0.0f;
+        float lb[4] = {0.0f, 0.0f, 0.0f, 0.0f}, zb[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // independent partial sums
 #pragma unroll
         for (int c = 0; c < kTcBlock / 8; ++c) {
             uint32_t hw[4], lw[4];
@@ -470,8 +487,8 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
                 const float2 v0 = sm.vsz[t0], v1 = sm.vsz[t0 + 1];
                 const float p0 = fast_exp2(fmaf(__uint_as_float(sc[t0]), qexp, cofs));
                 const float p1 = fast_exp2(fmaf(__uint_as_float(sc[t0 + 1]), qexp, cofs));
-                lb += p0 + p1;
-                Zs = fmaf(p0, v0.y, fmaf(p1, v1.y, Zs));
+                lb[e] += p0 + p1;
+                zb[e] = fmaf(p0, v0.y, fmaf(p1, v1.y, zb[e]));
                 const float a = p0 * v0.x, b = p1 * v1.x;
                 const __half2 hi2 = __floats2half2_rn(a, b);
                 const float2 back = __half22float2(hi2);
@@ -483,7 +500,8 @@ __global__ void __launch_bounds__(kTcRows, 2) extend_tc_kernel(const __grid_cons
             *reinterpret_cast<uint4*>(sm.p[0] + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             *reinterpret_cast<uint4*>(sm.p[1] + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
-        l += lb;
+        l += (lb[0] + lb[1]) + (lb[2] + lb[3]);
+        Zs += (zb[0] + zb[1]) + (zb[2] + zb[3]);
         ++since_fold;
         fence_proxy_async();
         tc_before_sync();
