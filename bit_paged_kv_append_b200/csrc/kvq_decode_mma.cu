@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         const uint8_t* st = R.stage[warp][slot];
         const uint32_t vmask = R.mask[warp][slot];
         const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
-        stage_szf<CB>(R, st, warp, lane, 1.0f);
+        stage_szf<CB>(R, st, warp, lane, 1.0f, kPScale);
 
         // ---- scores: q_int . codes for the two 8-token n-tiles (column gq: token 8 tau + tokK) ----
         float C[2][2];
@@ -260,9 +260,10 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
             float cm = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
             cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 1));
             cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 2));
-            const float mn = fmaxf(m, cm);
-            if (__any_sync(kFull, mn > m)) {
-                const float alpha = (mn > m) ? fast_exp2(m - mn) : 1.0f;
+            const bool up = cm > m + kTau;  // lazily moved reference (m = -inf: any finite cm)
+            const float mn = up ? cm : m;
+            if (__any_sync(kFull, up)) {
+                const float alpha = up ? fast_exp2(m - mn) : 1.0f;
                 l *= alpha;
                 Z *= alpha;
                 m = mn;
@@ -329,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         float v[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            v[2 * j] = O[j][0] * kTwo24 + Z0;
-            v[2 * j + 1] = O[j][2] * kTwo20 + Z0;
+            v[2 * j] = O[j][0] * (kTwo24 * kPOut) + Z0;
+            v[2 * j + 1] = O[j][2] * (kTwo20 * kPOut) + Z0;
         }
         mo_store16<G>(mo, warp * G + h0, h0, gq, v);
     }
@@ -338,8 +339,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_mma_kernel(DecodeParams p)
         float v[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            v[2 * j] = O[j][1] * kTwo24 + Z1;
-            v[2 * j + 1] = O[j][3] * kTwo20 + Z1;
+            v[2 * j] = O[j][1] * (kTwo24 * kPOut) + Z1;
+            v[2 * j + 1] = O[j][3] * (kTwo20 * kPOut) + Z1;
         }
         mo_store16<G>(mo, warp * G + h1, h1, gq, v);
     }
@@ -452,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         const uint8_t* st = R.stage[warp][slot];
         const uint32_t vmask = R.mask[warp][slot];
         const int tb = cs.t0 + (warp + kWarps * i) * kChunk;
-        stage_szf<CB>(R, st, warp, lane, 1.0f);
+        stage_szf<CB>(R, st, warp, lane, 1.0f, kPScale);
 
         // ---- scores: codes (tokens tk, tk + 8; bytes [16 pq, 16 pq + 16)) . q_int ----
         const uint4 k0 = key_codes<CB>(st, tk, pq);
@@ -479,9 +480,10 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 4));
         cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 8));
         cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 16));
-        const float mn = fmaxf(m, cm);
-        if (__any_sync(kFull, mn > m)) {
-            const float alpha = (mn > m) ? fast_exp2(m - mn) : 1.0f;
+        const bool up = cm > m + kTau;  // lazily moved reference (m = -inf: any finite cm)
+        const float mn = up ? cm : m;
+        if (__any_sync(kFull, up)) {
+            const float alpha = up ? fast_exp2(m - mn) : 1.0f;
             l *= alpha;
             Z *= alpha;
             m = mn;
@@ -537,8 +539,8 @@ __global__ void __launch_bounds__(kThreads, 5) decode_tok_kernel(DecodeParams p)
         float v[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            v[2 * j] = (O[j][0] + O[j][1]) * kTwo24 + Z;
-            v[2 * j + 1] = (O[j][2] + O[j][3]) * kTwo20 + Z;
+            v[2 * j] = (O[j][0] + O[j][1]) * (kTwo24 * kPOut) + Z;
+            v[2 * j + 1] = (O[j][2] + O[j][3]) * (kTwo20 * kPOut) + Z;
         }
         mo_store16<G>(mo, warp * G + pq, pq, gq, v);
         if (gq == 0) {

@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 3) extend_kernel(ExtendParams ep) {
         const uint8_t* st = R.stage[warp][slot];
         const uint32_t vmask = R.mask[warp][slot];
         const int tb = i * kChunk;
-        stage_szf<CB>(R, st, warp, lane, 1.0f);
+        stage_szf<CB>(R, st, warp, lane, 1.0f, 1.0f);
 
         // ---- q_int . codes: column gq of n-tile tau is token 8 tau + tokK ----
         int X[2][4], Y[2][4], W[2][4];

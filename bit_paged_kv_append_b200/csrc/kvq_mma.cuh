@@ -329,14 +329,24 @@ __device__ __forceinline__ void load_q_rotated(const DecodeParams& p, int64_t qr
 
 // Chunk's (scale, zero) words into floats, one word per lane (0..15 K, 16..31 V).
 // Values use centred codes c - 8, so their offset is zero + 8 scale; kscale
-// multiplies the key scales (exactly: a power of two).
+// multiplies the key scales and vscale the value scales (exactly: powers of two).
 template <int CB>
-__device__ __forceinline__ void stage_szf(CtaRing& R, const uint8_t* st, int warp, int lane, float kscale) {
+__device__ __forceinline__ void stage_szf(CtaRing& R, const uint8_t* st, int warp, int lane, float kscale,
+                                          float vscale) {
     const uint32_t w = reinterpret_cast<const uint32_t*>(st + Stage<CB>::kOffKs)[lane];
     const float sc = half_lo(w), zr = half_hi(w);
-    R.szf[warp][lane >> 4][lane & 15] = lane < 16 ? make_float2(sc * kscale, zr) : make_float2(sc, zr + 8.0f * sc);
+    R.szf[warp][lane >> 4][lane & 15] =
+        lane < 16 ? make_float2(sc * kscale, zr) : make_float2(sc * vscale, zr + 8.0f * sc);
     __syncwarp();
 }
+
+// Lazily moved softmax reference: a row's reference max moves only when a chunk's max
+// passes it by kTau (log2 units), so p = 2^(s - m) stays below 2^kTau and most chunks skip
+// the rescale of the accumulators.  The decode multiplies value scales by kPScale so that
+// p scale 2^-kTau <= scale stays inside fp16; its output undoes the factor (kPOut).
+constexpr float kTau = 8.0f;
+constexpr float kPScale = 1.0f / 256.0f;  // 2^-kTau
+constexpr float kPOut = 256.0f;
 
 // V codes of one chunk as P.V A operands: for each 16-dim tile jv, f(jv, a) with
 // a = A[16 dims x 16 tokens], tokens (tokA, tokB), (8 + tokA, 8 + tokB) from bytes
