@@ -82,6 +82,10 @@ HEADLINE = {"batch16": ("bdr128_k", kvq.KV_INT4_BDR, 128, False),
 _DECODE_SOURCES = ["kvq_decode_mma.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh", "kvq_internal.h"]
 KERNEL_SOURCES = {"append_kernel": ["kvq_append.cu", "kvq_common.cuh", "kvq_internal.h"],
                   "decode_tok_kernel": _DECODE_SOURCES, "decode_mma_kernel": _DECODE_SOURCES,
+                  "decode_bf16_kernel": ["kvq_decode_bf16.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh",
+                                         "kvq_internal.h"],
+                  "extend_tc_kernel": ["kvq_extend_tc.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh",
+                                       "kvq_internal.h"],
                   "extend_kernel": ["kvq_extend.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh",
                                     "kvq_internal.h"]}
 
@@ -370,15 +374,17 @@ def run_extend(w: Workload, mode, b, rv, reps, device):
     per_tok = w.H * (2 * 68 if mode != kvq.KV_BF16 else 2 * 256)
     nbytes = sum(lens) * per_tok + nq * w.Hq * 128 * 2 * 2
     peak, kind = peak_bf16_tflops()
+    ekern = "extend_tc_kernel"  # 4-bit codes run on tcgen05 (2-bit codes would take extend_kernel, mma.sync)
     t = float(ms.mean())
     return {"us": t * 1e3, "us_median": float(np.median(ms)) * 1e3, "launches": reps, "sequences": len(seqs),
             "queries": nq, "query_heads": w.Hq, "attended_tokens_per_query_head": attended,
             "flops": flops, "tflops": flops / (t / 1e3) / 1e12,
-            "roofline": {"bound": "tensor", "kernel": "extend_kernel", "achieved": flops / (t / 1e3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": ekern, "achieved": flops / (t / 1e3) / 1e12,
                          "peak": peak, "unit": "TFLOP/s", "frac": flops / (t / 1e3) / 1e12 / peak,
-                         "peak_source": f"{kind} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops); the kernel "
-                                        "runs int8 (q.K) and fp16 (P.V) mma.sync tiles",
-                         "traffic": profiled_traffic("extend_kernel", w.name)},
+                         "peak_source": f"{kind} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops); " + (
+                             "the kernel runs fp16 tcgen05 MMAs (kind::f16, the same dense rate as bf16)"
+                             if ekern == "extend_tc_kernel" else "the kernel runs int8 (q.K) and fp16 (P.V) mma.sync tiles"),
+                         "traffic": profiled_traffic(ekern, w.name)},
             "algorithmic_bytes": nbytes, "gbs": nbytes / (t / 1e3) / 1e9,
             "device_status": kvq.status_string(status)}
 
@@ -603,7 +609,7 @@ CONFIG_STEPS = 50  # timed steps of each sub-record variant (after 3 warm-ups)
 
 def _dec_kernel(w: Workload, mode):
     if mode == kvq.KV_BF16:
-        return "bf16_split_kernel + merge_kernel"
+        return "decode_bf16_kernel + merge_kernel"
     # the INT4 decode runs the tokens-on-M tile for up to 4 query heads per KV head, else heads-on-M
     return ("decode_tok_kernel" if w.Hq // w.H <= 4 else "decode_mma_kernel") + " + merge_kernel"
 
@@ -714,6 +720,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-accuracy", action="store_true")
     ap.add_argument("--no-extend", action="store_true")
+    ap.add_argument("--extend-only", action="store_true",
+                    help="only the extend attention of --workload (3 warm-up + 10 timed launches), one JSON line; "
+                         "the entry point of its ncu captures")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -731,6 +740,15 @@ def main():
     w = Workload(args.workload, args.seed + rank, device)  # each rank: its own independent batch
     hname, hmode, hb, hrv = HEADLINE[args.workload]
     peak, peak_kind = peak_hbm()
+    if args.extend_only:
+        if extend_setup(w) is None:
+            raise SystemExit(f"{args.workload} has no prefill queries")
+        r = run_extend(w, hmode, hb, hrv, 10, device)
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, "variant": hname, "extend": r}))
+        if _dist is not None:
+            _dist.destroy_process_group()
+        return
 
     res = run_variant(w, hmode, hb, hrv, args.steps, args.warmup, device, clocks=True)
     res["steps"] = args.steps
