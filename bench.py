@@ -389,6 +389,38 @@ def run_extend(w: Workload, mode, b, rv, reps, device):
             "device_status": kvq.status_string(status)}
 
 
+def run_profile_case(case: str):
+    """Small seeded cases for ncu captures with many passes (more than L2 on the device, well under
+    1 GB): the cache is filled through the append, then the captured kernel runs 4 times."""
+    device = torch.device("cuda")
+    B, L, H, Hq, rv = (32, 4096, 8, 64, True) if case == "decode_g8" else (4, 4096, 8, 32, False)
+    ps = 16
+    num_pages = B * L // ps
+    g = torch.Generator(device=device).manual_seed(0)
+    pt = torch.randperm(num_pages, device=device, generator=g).to(torch.int32).view(B, L // ps).contiguous()
+    cache = kvq.PagedKVCache(num_pages, ps, H, Hq, kvq.KV_INT4_BDR, 128, rv, device=device, fill=0)
+    k = torch.randn(B * L, H, 128, device=device, generator=g).to(torch.bfloat16)
+    v = torch.randn(B * L, H, 128, device=device, generator=g).to(torch.bfloat16)
+    ts = torch.arange(B, device=device, dtype=torch.int32).repeat_interleave(L)
+    tp = torch.arange(L, device=device, dtype=torch.int32).repeat(B)
+    cache.append(k, v, ts, tp, pt)
+    sl = torch.full((B,), L, device=device, dtype=torch.int32)
+    if case == "decode_g8":
+        q = torch.randn(B, Hq, 128, device=device, generator=g).to(torch.bfloat16)
+        ws = cache.workspace(B, L, device)
+        for _ in range(4):
+            out = cache.decode(q, sl, pt, L, workspace=ws)
+    else:
+        q = torch.randn(B * L, Hq, 128, device=device, generator=g).to(torch.bfloat16)
+        qi = torch.arange(0, B * L + 1, L, device=device, dtype=torch.int32)
+        for _ in range(4):
+            out = cache.extend(q, qi, sl, pt, L, L)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": case, "sequences": B, "tokens_per_sequence": L, "num_kv_heads": H,
+                      "num_q_heads": Hq, "device_status": kvq.status_string(cache.get_error()),
+                      "mean_abs_out": float(out.float().abs().mean())}))
+
+
 def exact_attention(k, v, q, lengths, H, Hq):
     """float64 attention of q over the unquantised bf16 K/V rows (sequence-major, positions 0..L-1):
     the values the quantised caches approximate (no cache, no quantisation, no rotation)."""
@@ -720,11 +752,19 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-accuracy", action="store_true")
     ap.add_argument("--no-extend", action="store_true")
+    ap.add_argument("--profile-case", choices=["decode_g8", "extend_g4"],
+                    help="a small case for multi-metric ncu captures: decode_g8 = 32 sequences x 4096 tokens, "
+                         "64 query / 8 KV heads, BDR-128 keys and values, 4 decode launches; extend_g4 = 4 "
+                         "sequences x 4096 tokens, 32 query / 8 KV heads, BDR-128 keys, full causal prefill, "
+                         "4 extend launches")
     ap.add_argument("--extend-only", action="store_true",
                     help="only the extend attention of --workload (3 warm-up + 10 timed launches), one JSON line; "
                          "the entry point of its ncu captures")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    if args.profile_case:
+        return run_profile_case(args.profile_case)
 
     if args.impl == "reference":
         # the CPU oracle: rank 0 alone runs it, other ranks exit without work
