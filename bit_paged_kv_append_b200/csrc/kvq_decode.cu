@@ -130,6 +130,9 @@ DecodePlan plan_decode(const CacheGeom& g, int batch, int max_seq_len, int num_s
     int64_t it = (int64_t(batch) * g.H * L * 4 + 11 * slots - 1) / (11 * slots);
     it = ((it + 63) / 64) * 64;
     if (it < 512) it = 512;
+    // BF16 pages move 4 KiB a token and their split kernel holds 2 CTAs per SM: splits of at
+    // least 2048 tokens (measured: batch16 40.0 -> 37.8 us, the long workloads unchanged)
+    if (g.mode == 0 && it < 2048) it = 2048;
     if (it > 4096) it = 4096;
     pl.item_tokens = int(it);
     pl.max_splits = int((L + it - 1) / it);
