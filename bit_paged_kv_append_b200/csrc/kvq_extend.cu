@@ -425,7 +425,7 @@ cudaError_t launch_k(const ExtendParams& ep, dim3 grid, cudaStream_t s) {
 
 template <int G>
 cudaError_t launch_group(const ExtendParams& ep, dim3 grid, cudaStream_t s) {
-    return ep.d.g.code_bits == 2 ? launch_k<G, 2>(ep, grid, s) : launch_k<G, 4>(ep, grid, s);
+    return launch_k<G, 2>(ep, grid, s);  // only 2-bit codes reach this kernel
 }
 
 }  // namespace
