@@ -12,7 +12,7 @@
 // so both contractions run on raw 4-bit codes.
 //
 // One CTA = 128 (query, head) rows of one KV head of one sequence (128 / G consecutive
-// queries x the G heads), one CTA per SM (206 KB of shared memory, all 512 TMEM columns),
+// queries x the G heads), one CTA per SM (207 KB of shared memory, all 512 TMEM columns),
 // three warp roles working on blocks of 128 key tokens:
 //   * loaders (warps 8-11, thread = token): gather a block's key and value code rows through
 //     the page table and write them as fp16 operand tiles: key codes as the exact
@@ -32,9 +32,9 @@
 //     that keeps P below 2^15) as fp16 high and low parts over S_j in TMEM.
 // The softmax of block j overlaps q.K of block j + 1 and P.V of block j - 1.  The tensor
 // cores' fp32 accumulation does not round to nearest, and over thousands of tokens its bias
-// would grow: O_t runs at most 4 blocks (512 tokens), then the softmax folds it into an fp32
-// copy O_f in shared memory with ordinary adds (and rescales O_f when a row's reference
-// moves), and the next P.V restarts O_t.  Both operands of q.K in shared memory would take
+// would grow: O_t runs 4 blocks (512 tokens), then the softmax folds it into an fp32 copy O_f
+// in shared memory with ordinary adds and the next P.V restarts O_t; a row whose reference
+// moves rescales its part of O_t in place and of O_f.  Both operands of q.K in shared memory would take
 // ~120 B per clock, the whole shared-memory port, while the softmax and the loaders need it
 // too; with q in tensor memory q.K reads only the key tiles.
 //
@@ -53,7 +53,7 @@ constexpr int kXBlk = 128;    // key tokens per block = loader threads
 constexpr int kXSoftWarps = 8, kXLoadWarps = 4;
 constexpr int kXSoftThreads = 32 * kXSoftWarps;  // two per row
 constexpr int kXMmaWarp = kXSoftWarps + kXLoadWarps;
-constexpr int kXThreads = 32 * (kXMmaWarp + 1);
+constexpr int kXThreads = 32 * (kXMmaWarp + 4);  // the MMA warp's warpgroup: the issuer + 3 idle warps
 constexpr int kXCols = 512;                  // TMEM columns: S_0 | S_1 | O_t | q' (high, low)
 constexpr uint32_t kColS = 0, kColOt = 256, kColQ = 384;
 constexpr int kFoldEvery = 4;                // blocks accumulated in O_t between folds (512 tokens)
@@ -152,12 +152,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t* v) {
         : "memory");
 }
 
-// Register split (per thread): the launch gives 128 to each of the 13 warps (four warps share
-// scheduler 0).  The two softmax warpgroups raise their share to 160 once the loader warpgroup
-// has lowered its own to 64; the MMA warp keeps 128.  8 x 32 x 160 + 4 x 32 x 64 + 32 x 128 =
-// 53248 = 416 x 128, the launch's total, so the raise never waits for registers that do not exist.
-constexpr int kXRegsSoft = 160, kXRegsLoad = 64, kXRegsLaunch = 128;
-static_assert(kXSoftThreads * kXRegsSoft + 32 * kXLoadWarps * kXRegsLoad + 32 * kXRegsLaunch <=
+// Register split (per thread): the launch gives 128 to each of the 16 warps (four per
+// scheduler).  The loader warpgroup lowers its share to 104 and the MMA warpgroup (the
+// issuing warp and three idle ones, there so that the group can give registers back) to
+// 40; the two softmax warpgroups then raise theirs to 184.  8 x 32 x 184 + 4 x 32 x 104 +
+// 4 x 32 x 40 = 65536 = 512 x 128, the launch's total, so the raise never waits for
+// registers that do not exist (and no role spills).
+constexpr int kXRegsSoft = 184, kXRegsLoad = 104, kXRegsMma = 40, kXRegsLaunch = 128;
+static_assert(kXSoftThreads * kXRegsSoft + 32 * kXLoadWarps * kXRegsLoad + 128 * kXRegsMma <=
                   kXThreads * kXRegsLaunch,
               "register split exceeds the launch's registers");
 
@@ -724,6 +726,7 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
         cta_bar();
     } else {
         // =============================== MMA issue ===============================
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kXRegsMma));
         cta_bar();  // barriers initialised
         cta_bar();  // q tiles, tensor memory, row lengths
         tc_after_sync();
@@ -731,7 +734,7 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
         const int nblocks = (sm.tmax + kXBlk - 1) / kXBlk;
         grid_dep_wait();
         grid_dep_launch();
-        if (lane == 0) {
+        if (warp == kXMmaWarp && lane == 0) {
             bool issued = false;
             for (int j = 0; j <= nblocks; ++j) {
                 if (*abort) break;
