@@ -413,14 +413,14 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
             float mb4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             const float4* kz4 = reinterpret_cast<const float4*>(sm.ksz[b]) + 32 * hf;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {  // 16 tokens at a time: their 8 (scale, zero) loads issue together
-                float4 kz[8];
+            for (int c = 0; c < 2; ++c) {  // 32 tokens at a time: their 16 (scale, zero) loads issue together
+                float4 kz[16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) kz[i] = kz4[8 * c + i];
-                const uint32_t vm = full ? 0xFFFFFFFFu : sm.vmask[b][2 * hf + (c >> 1)] >> (16 * (c & 1));
+                for (int i = 0; i < 16; ++i) kz[i] = kz4[16 * c + i];
+                const uint32_t vm = full ? 0xFFFFFFFFu : sm.vmask[b][2 * hf + c];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int t = 16 * c + 2 * i;
+                for (int i = 0; i < 16; ++i) {
+                    const int t = 32 * c + 2 * i;
                     const float v0 = fmaf(kz[i].x, __uint_as_float(sv[t]), zq * kz[i].y);
                     const float v1 = fmaf(kz[i].z, __uint_as_float(sv[t + 1]), zq * kz[i].w);
                     const float m0 = (full || ((tb + t < rowlen) && ((vm >> (2 * i)) & 1u))) ? v0 : -INFINITY;
@@ -504,14 +504,14 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
             const float4* vz4 = reinterpret_cast<const float4*>(sm.vsz[b]) + 32 * hf;
             float lb[4] = {0.0f, 0.0f, 0.0f, 0.0f}, zb[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // independent partial sums
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {  // 16 tokens at a time
-                uint32_t hw[8], lw[8];
-                float4 vzc[8];  // their 8 (scale, zero + 8 scale) loads issue together
+            for (int c = 0; c < 2; ++c) {  // 32 tokens (chunk 2 hf + c of the block) at a time
+                uint32_t hw[16], lw[16];
+                float4 vzc[16];  // their 16 (scale, zero + 8 scale) loads issue together
 #pragma unroll
-                for (int i = 0; i < 8; ++i) vzc[i] = vz4[8 * c + i];
+                for (int i = 0; i < 16; ++i) vzc[i] = vz4[16 * c + i];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int t0 = 16 * c + 2 * e;
+                for (int e = 0; e < 16; ++e) {
+                    const int t0 = 32 * c + 2 * e;
                     const float4 vz = vzc[e];
                     const float p0 = fast_exp2(fmaf(__uint_as_float(sv[t0]), qexp, cofs));
                     const float p1 = fast_exp2(fmaf(__uint_as_float(sv[t0 + 1]), qexp, cofs));
@@ -525,9 +525,9 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
                     lw[e] = *reinterpret_cast<const uint32_t*>(&lo2);
                 }
                 // tokens 16 c .. 16 c + 15 of this half: chunk 2 hf + c / 2 of the block, its (c % 2)-th 8 pairs
-                const uint32_t pc = s_col + 64 * hf + 32 * (c >> 1) + 8 * (c & 1);
-                tmem_st8(pc, hw);
-                tmem_st8(pc + 16, lw);
+                const uint32_t pc = s_col + 64 * hf + 32 * c;
+                tmem_st16(pc, hw);
+                tmem_st16(pc + 16, lw);
             }
             l += (lb[0] + lb[1]) + (lb[2] + lb[3]);
             Zs += (zb[0] + zb[1]) + (zb[2] + zb[3]);
