@@ -57,6 +57,7 @@ CASES = [  # (id, H, Hq, page size, mode, block, rotate_v, code bits)
     ("g8_bdr128kv", 2, 16, 16, kvq.KV_INT4_BDR, 128, True, 4),
     ("g4_int4_ps7", 2, 8, 7, kvq.KV_INT4, 0, False, 4),
     ("g1_bdr64kv", 4, 4, 16, kvq.KV_INT4_BDR, 64, True, 4),
+    ("g2_bdr128kv_ps32", 4, 8, 32, kvq.KV_INT4_BDR, 128, True, 4),
     ("g2_bdr32k_int2", 2, 4, 16, kvq.KV_INT4_BDR, 32, False, 2),
     ("g8_bdr16kv_int2_ps12", 1, 8, 12, kvq.KV_INT4_BDR, 16, True, 2),
 ]
