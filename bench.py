@@ -85,9 +85,7 @@ KERNEL_SOURCES = {"append_kernel": ["kvq_append.cu", "kvq_common.cuh", "kvq_inte
                   "decode_bf16_kernel": ["kvq_decode_bf16.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh",
                                          "kvq_internal.h"],
                   "extend_tc_kernel": ["kvq_extend_tc.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh",
-                                       "kvq_internal.h"],
-                  "extend_kernel": ["kvq_extend.cu", "kvq_mma.cuh", "kvq_decode.cuh", "kvq_common.cuh",
-                                    "kvq_internal.h"]}
+                                       "kvq_internal.h"]}
 
 
 def peak_bf16_tflops():
@@ -374,7 +372,7 @@ def run_extend(w: Workload, mode, b, rv, reps, device):
     per_tok = w.H * (2 * 68 if mode != kvq.KV_BF16 else 2 * 256)
     nbytes = sum(lens) * per_tok + nq * w.Hq * 128 * 2 * 2
     peak, kind = peak_bf16_tflops()
-    ekern = "extend_tc_kernel"  # 4-bit codes run on tcgen05 (2-bit codes would take extend_kernel, mma.sync)
+    ekern = "extend_tc_kernel"
     t = float(ms.mean())
     return {"us": t * 1e3, "us_median": float(np.median(ms)) * 1e3, "launches": reps, "sequences": len(seqs),
             "queries": nq, "query_heads": w.Hq, "attended_tokens_per_query_head": attended,
@@ -382,8 +380,7 @@ def run_extend(w: Workload, mode, b, rv, reps, device):
             "roofline": {"bound": "tensor", "kernel": ekern, "achieved": flops / (t / 1e3) / 1e12,
                          "peak": peak, "unit": "TFLOP/s", "frac": flops / (t / 1e3) / 1e12 / peak,
                          "peak_source": f"{kind} dense bf16 burst (MEASURED_PEAKS.json bf16_tflops); " + (
-                             "the kernel runs fp16 tcgen05 MMAs (kind::f16, the same dense rate as bf16)"
-                             if ekern == "extend_tc_kernel" else "the kernel runs int8 (q.K) and fp16 (P.V) mma.sync tiles"),
+                             "the kernel runs fp16 tcgen05 MMAs (kind::f16, the same dense rate as bf16)"),
                          "traffic": profiled_traffic(ekern, w.name)},
             "algorithmic_bytes": nbytes, "gbs": nbytes / (t / 1e3) / 1e9,
             "device_status": kvq.status_string(status)}

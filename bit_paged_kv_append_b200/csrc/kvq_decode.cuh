@@ -76,8 +76,5 @@ __device__ __forceinline__ float fast_exp2(float x) {  // MUFU ex2; exp2(-inf) =
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s);
 // Tensor-core split kernel for BF16 pages (grid: max_splits x H x B).
 cudaError_t launch_decode_bf16(const DecodeParams& p, cudaStream_t s);
-// Extend attention on tcgen05 for 4-bit codes (kvq_extend_tc.cu): p carries the cache, q,
-// seq_lens, page table, output and error word; q_indptr [batch + 1] marks each sequence's queries.
-cudaError_t launch_extend_tc(const DecodeParams& p, const int32_t* q_indptr, int max_q_len, cudaStream_t s);
 
 }  // namespace kvq

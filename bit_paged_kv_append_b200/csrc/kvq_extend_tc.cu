@@ -1,5 +1,5 @@
-// kvq_extend_tc.cu -- extend (chunked-prefill) attention over the paged INT4 cache on the
-// 5th-generation tensor cores (tcgen05.mma, operands and accumulators in tensor memory).
+// kvq_extend_tc.cu -- extend (chunked-prefill) attention over the paged INT4 (or 2-bit) cache
+// on the 5th-generation tensor cores (tcgen05.mma, operands and accumulators in tensor memory).
 //
 // SAW-INT4's abstract keeps fused attention over the paged quantised layout as a serving
 // constraint; chunked prefill in mixed serving reads the cache this way.  Query i of the n
@@ -16,8 +16,9 @@
 // three warp roles working on blocks of 128 key tokens:
 //   * loaders (warps 8-11, thread = token): gather a block's key and value code rows through
 //     the page table and write them as fp16 operand tiles: key codes as the exact
-//     subnormals c 2^-24 (B of q.K, K-major), value codes centred, (c - 8) 2^-24 (B of P.V,
-//     N-major), with the tokens' scales and zeros.  Two stages; the key tile is released
+//     subnormals c 2^-24 (B of q.K, K-major), value codes centred, (c - 8) 2^-24 for 4-bit
+//     codes and (c - 2) 2^-24 for 2-bit ones (B of P.V, N-major), with the tokens' scales and
+//     zeros.  2-bit rows (32 bytes) are first spread to the 4-bit nibble layout.  Two stages; the key tile is released
 //     when its q.K is done, the value tile when its P.V is done;
 //   * one MMA thread (warp 12): S_j[128 x 128] = q_hi K_j^T + q_lo K_j^T (16 MMAs M128 N128
 //     K16, kind::f16, q read from TMEM, the key tile from shared memory) into one of two TMEM
@@ -41,8 +42,7 @@
 // Every mbarrier wait is bounded (kWaitLimitNs, and it gives up early once another role has
 // given up); on expiry the CTA flags KV_ERR_TIMEOUT, each role leaves its loop, the MMA
 // thread waits (bounded) for every MMA it issued, and the tensor memory is freed.  No
-// hardware barrier is entered by only part of its threads.  The 2-bit variant keeps the
-// mma.sync kernel (kvq_extend.cu).
+// hardware barrier is entered by only part of its threads.
 #include "kvq_mma.cuh"
 
 namespace kvq {
@@ -139,11 +139,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t* v) {
           "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
         : "r"(addr));
 }
-__device__ __forceinline__ void tmem_st8(uint32_t addr, const uint32_t* v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(addr), "r"(v[0]),
-                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
-}
 __device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t* v) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::
@@ -221,10 +216,14 @@ __device__ __forceinline__ void codes_to_f16(uint32_t w, uint32_t centre, uint32
     }
 }
 
-template <int G>
+template <int G, int CB>
 __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant__ DecodeParams p,
                                                                  const int32_t* __restrict__ q_indptr, int max_q_len) {
     constexpr int QB = kXRows / G;  // queries per CTA
+    // value codes are centred at the middle of their range: c - 8 (4-bit) or c - 2 (2-bit)
+    constexpr float kCentre = CB == 4 ? 8.0f : 2.0f;
+    constexpr uint32_t kCentreF16 = CB == 4 ? kMinus8 : 0x80028002u;  // fp16x2 (-centre 2^-24, -centre 2^-24)
+    constexpr uint32_t kCentreNib = CB == 4 ? 0x88888888u : 0x22222222u;  // every nibble at the centre
     extern __shared__ uint8_t dsm_raw[];
     XSmem& sm = *reinterpret_cast<XSmem*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
     volatile int* abort = &sm.abort;
@@ -648,23 +647,38 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
             const int T = j * kXBlk + t;
             const int page = npage;
             npage = page_id(j + 1);
-            uint4 ck[4], cv[4];
+            // the token's key and value codes as 16 words of the 4-bit nibble layout (word n: dims
+            // 8 n .. 8 n + 7); a masked token's values are the centre itself (centred zero)
+            uint32_t nk[16], nv[16];
             uint32_t cks = 0, cvs = 0;
             bool tok = false;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                ck[i] = make_uint4(0u, 0u, 0u, 0u);
-                cv[i] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);  // centred zero
+            for (int n = 0; n < 16; ++n) {
+                nk[n] = 0u;
+                nv[n] = kCentreNib;
             }
             if (T < tmax) {
                 if (page >= 0 && page < p.g.num_pages) {
                     const int64_t row = (int64_t(page) * p.g.H + h) * p.g.page_size + slot_of_pos(p, T);
-                    const uint4* kr = reinterpret_cast<const uint4*>(kpool + row * 64);
-                    const uint4* vr = reinterpret_cast<const uint4*>(vpool + row * 64);
+                    const uint4* kr = reinterpret_cast<const uint4*>(kpool + row * (16 * CB));
+                    const uint4* vr = reinterpret_cast<const uint4*>(vpool + row * (16 * CB));
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        ck[i] = __ldg(kr + i);
-                        cv[i] = __ldg(vr + i);
+                    for (int i = 0; i < CB; ++i) {  // 16-byte units of the row: 4 (4-bit) or 2 (2-bit)
+                        const uint4 a = __ldg(kr + i), c = __ldg(vr + i);
+                        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            if (CB == 4) {
+                                nk[4 * i + e] = aw[e];
+                                nv[4 * i + e] = cw[e];
+                            } else {  // 16 two-bit codes (dims 16 m .. 16 m + 15) -> two nibble words
+                                const uint2 ka = expand2(aw[e]), va = expand2(cw[e]);
+                                nk[8 * i + 2 * e] = ka.x;
+                                nk[8 * i + 2 * e + 1] = ka.y;
+                                nv[8 * i + 2 * e] = va.x;
+                                nv[8 * i + 2 * e + 1] = va.y;
+                            }
+                        }
                     }
                     cks = __ldg(p.g.k_sz + row);
                     cvs = __ldg(p.g.v_sz + row);
@@ -681,14 +695,10 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
             }
             if (!w) break;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t kw[4] = {ck[i].x, ck[i].y, ck[i].z, ck[i].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    uint32_t o4[4];
-                    codes_to_f16(kw[e], 0u, o4);
-                    *reinterpret_cast<uint4*>(sm.k[b] + tile_off(t, 32 * i + 8 * e)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-                }
+            for (int n = 0; n < 16; ++n) {
+                uint32_t o4[4];
+                codes_to_f16(nk[n], 0u, o4);
+                *reinterpret_cast<uint4*>(sm.k[b] + tile_off(t, 8 * n)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
             fence_proxy_async();
             mbar_arrive(&sm.k_full[b]);
@@ -699,19 +709,15 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
             }
             if (!w) break;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t vw[4] = {cv[i].x, cv[i].y, cv[i].z, cv[i].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    uint32_t o4[4];
-                    codes_to_f16(vw[e], kMinus8, o4);
-                    *reinterpret_cast<uint4*>(sm.v[b] + tile_off(t, 32 * i + 8 * e)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-                }
+            for (int n = 0; n < 16; ++n) {
+                uint32_t o4[4];
+                codes_to_f16(nv[n], kCentreF16, o4);
+                *reinterpret_cast<uint4*>(sm.v[b] + tile_off(t, 8 * n)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
             const float ksc = half_lo(cks), kzr = half_hi(cks);
             const float vsc = half_lo(cvs), vzr = half_hi(cvs);
             sm.ksz[b][t] = tok ? make_float2(ksc, kzr) : make_float2(0.0f, 0.0f);
-            sm.vsz[b][t] = tok ? make_float2(vsc, vzr + 8.0f * vsc) : make_float2(0.0f, 0.0f);
+            sm.vsz[b][t] = tok ? make_float2(vsc, vzr + kCentre * vsc) : make_float2(0.0f, 0.0f);
             float vmx = tok ? fabsf(vsc) : 0.0f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) vmx = fmaxf(vmx, __shfl_xor_sync(0xffffffffu, vmx, o));
@@ -784,27 +790,46 @@ __global__ void __maxnreg__(kXRegsLaunch) extend_tc_kernel(const __grid_constant
     }
 }
 
-template <int G>
+template <int G, int CB>
 cudaError_t launch_g(const DecodeParams& dp, const int32_t* q_indptr, int max_q_len, dim3 grid, cudaStream_t s) {
-    constexpr auto kern = extend_tc_kernel<G>;
+    constexpr auto kern = extend_tc_kernel<G, CB>;
     const cudaError_t e = ensure_smem_opt_in<kern>(kXSmem);
     if (e != cudaSuccess) return e;
     return launch_overlapped(kern, grid, dim3(kXThreads), kXSmem, s, dp, q_indptr, max_q_len);
 }
 
-}  // namespace
-
-cudaError_t launch_extend_tc(const DecodeParams& dp, const int32_t* q_indptr, int max_q_len, cudaStream_t s) {
-    const int G = dp.g.Hq / dp.g.H;
-    const int qb = kXRows / G;
-    const dim3 grid((max_q_len + qb - 1) / qb, dp.g.H, dp.a.batch);
-    switch (G) {
-        case 1: return launch_g<1>(dp, q_indptr, max_q_len, grid, s);
-        case 2: return launch_g<2>(dp, q_indptr, max_q_len, grid, s);
-        case 4: return launch_g<4>(dp, q_indptr, max_q_len, grid, s);
-        case 8: return launch_g<8>(dp, q_indptr, max_q_len, grid, s);
+template <int CB>
+cudaError_t launch_cb(const DecodeParams& dp, const int32_t* q_indptr, int max_q_len, dim3 grid, cudaStream_t s) {
+    switch (dp.g.Hq / dp.g.H) {
+        case 1: return launch_g<1, CB>(dp, q_indptr, max_q_len, grid, s);
+        case 2: return launch_g<2, CB>(dp, q_indptr, max_q_len, grid, s);
+        case 4: return launch_g<4, CB>(dp, q_indptr, max_q_len, grid, s);
+        case 8: return launch_g<8, CB>(dp, q_indptr, max_q_len, grid, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+}  // namespace
+
+cudaError_t launch_extend(const CacheGeom& g, const ExtendArgs& a, int* err_word, cudaStream_t s) {
+    if (a.batch == 0 || a.max_q_len == 0) return cudaSuccess;
+    DecodeParams dp;
+    dp.g = g;
+    dp.a = DecodeArgs{a.q, a.seq_lens, a.page_table, a.pt_stride, a.batch, a.max_seq_len, a.out, a.out_fp32,
+                      nullptr, 0};
+    dp.item_tokens = 0;
+    dp.max_splits = 0;
+    dp.qscale = float(1.0 / sqrt(double(kHeadDim))) * kLog2e;
+    dp.ps_shift = -1;
+    for (int sh = 0; sh < 11; ++sh)
+        if ((1 << sh) == g.page_size) dp.ps_shift = sh;
+    dp.ws_o = nullptr;
+    dp.ws_ml = nullptr;
+    dp.err = err_word;
+    const int qb = kXRows / (g.Hq / g.H);
+    const dim3 grid((a.max_q_len + qb - 1) / qb, g.H, a.batch);
+    return g.code_bits == 2 ? launch_cb<2>(dp, a.q_indptr, a.max_q_len, grid, s)
+                            : launch_cb<4>(dp, a.q_indptr, a.max_q_len, grid, s);
 }
 
 }  // namespace kvq

@@ -73,10 +73,8 @@ DecodePlan plan_decode(const CacheGeom& g, int batch, int max_seq_len, int num_s
 cudaError_t launch_append(const CacheGeom& g, const AppendArgs& a, int* err_word, int num_sms, cudaStream_t s);
 cudaError_t launch_decode(const CacheGeom& g, const DecodeArgs& a, const DecodePlan& plan, int* err_word,
                           cudaStream_t s);
-// INT4 modes only (the caller rejects BF16 pages).
+// INT4 modes only (the caller rejects BF16 pages); kvq_extend_tc.cu.
 cudaError_t launch_extend(const CacheGeom& g, const ExtendArgs& a, int* err_word, cudaStream_t s);
-// Query rows one extend CTA covers for this cache (grid extent along the queries: max_q_len / this).
-int extend_queries_per_cta(const CacheGeom& g);
 
 // Makes the handle's device current for the duration of one C-ABI call (and restores the
 // caller's device afterwards), so that launches, function attributes and symbol lookups

@@ -1,5 +1,6 @@
 // kvq_mma.cuh -- what the tensor-core attention kernels over the INT4 cache share
-// (decode in kvq_decode_mma.cu, extend in kvq_extend.cu): mma.sync wrappers, the
+// (decode in kvq_decode_mma.cu and kvq_decode_bf16.cu; the extend in kvq_extend_tc.cu takes
+// the rotated query loader's constants and the 2-bit spreading): mma.sync wrappers, the
 // per-warp ring of 16-token chunk stages and its cp.async copies, the rotated query,
 // the 23-bit fixed-point q digits, the key-code B fragments and the V-code A tiles.
 //
