@@ -105,3 +105,25 @@ def test_reference_arm_prints_the_kernel_arms_config(capsys):
     assert kw["row_budget"] == w.Hq and kw["reps"] >= 3
     assert f"decode of {w.Hq} query-head rows" in line["cpu_baseline"]["sample"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_kernel_source_lists_and_profiled_traffic_are_consistent():
+    """Every source a benched kernel's counters are keyed on exists; every profiled-traffic entry
+    names a benched kernel, and its hash is what src_hash gives now (or the bench reports null)."""
+    import json
+    import os
+
+    csrc = os.path.join(bench.ROOT, "bit_paged_kv_append_b200", "csrc")
+    for kernel, files in bench.KERNEL_SOURCES.items():
+        for name in files:
+            assert os.path.isfile(os.path.join(csrc, name)), (kernel, name)
+        assert len(bench.src_hash(kernel)) == 16
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        traffic = json.load(f)
+    for kernel, recs in traffic.items():
+        assert kernel in bench.KERNEL_SOURCES, kernel
+        for workload, rec in recs.items():
+            assert workload in synth.WORKLOADS, workload
+            assert rec["dram_bytes_per_launch"] == rec["dram_read"] + rec["dram_write"]
+            expect = float(rec["dram_bytes_per_launch"]) if rec["src_sha"] == bench.src_hash(kernel) else None
+            assert bench.profiled_traffic(kernel, workload) == expect
