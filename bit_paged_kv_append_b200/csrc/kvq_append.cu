@@ -25,9 +25,16 @@
 // sub-partition, so a thread may hold ~200 registers) read their row from the
 // swizzled stage without bank conflicts, write 64 B of codes + 4 B of (scale,
 // zero) per row straight to the pool, and free the stage on an mbarrier: no
-// block-wide barrier in the loop.  A tile = 224 consecutive rows of the
-// [T, H, D] input = 224 / H tokens (H divides 32); its K rows fill one stage and
-// its V rows the next.
+// block-wide barrier in the loop.  A tile = up to 224 consecutive rows of the
+// [T, H, D] input = up to 224 / H tokens (H divides 32); its K rows fill one stage
+// and its V rows the next.
+//
+// Schedule: CTA c owns the contiguous chunk of ceil(T / SMs) tokens starting at
+// c * that, so no CTA holds more than one token above the mean.  A chunk that is
+// not a whole number of tiles starts with its remainder as one short tile, copied
+// by a second pair of tensor maps whose box is that remainder's rows, then whole
+// tiles: with 4.01 tiles of work per SM every CTA runs four whole tiles and one
+// short one, not two CTAs five whole ones.
 //
 // Every wait is bounded (kWaitLimitNs); out-of-range sequence ids, positions
 // and page ids are skipped and flagged in the device error word.
@@ -72,11 +79,24 @@ constexpr uint32_t kMagicPackOffset2 = magic_pack_offset2();
 struct Params {
     CacheGeom g;
     AppendArgs a;
-    int num_tiles;
-    int tile_tokens;  // kRows / H
-    float r_b;        // (float)(1 / sqrt((double)bdr_block))
+    int tile_tokens;   // kRows / H: tokens of a whole tile
+    int chunk_tokens;  // tokens per CTA (the last CTA's chunk may be shorter)
+    int short_tokens;  // tokens the short-tile maps' box covers (0: no short maps)
+    float r_b;         // (float)(1 / sqrt((double)bdr_block))
     int* err;
 };
+
+struct Tile {
+    int first, count;  // first token, tokens (count 0: past the end of the chunk)
+};
+
+// Tile j of the chunk [c0, c0 + len): the remainder len % TT first, then whole tiles.
+__device__ __forceinline__ Tile tile_of(int c0, int len, int TT, int j) {
+    const int rem = len % TT;
+    const int first = rem ? (j == 0 ? c0 : c0 + rem + (j - 1) * TT) : c0 + j * TT;
+    const int count = (rem && j == 0) ? rem : TT;
+    return first < c0 + len ? Tile{first, count} : Tile{0, 0};
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -360,7 +380,8 @@ __device__ __forceinline__ void copy_row(const uint8_t* stage, int row, uint8_t*
 
 template <int MODE, int BLK, bool ROTV, bool ROPE, int CB>
 __global__ void __launch_bounds__(kThreads, 1)
-    append_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, Params p) {
+    append_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                  const __grid_constant__ CUtensorMap kmap_s, const __grid_constant__ CUtensorMap vmap_s, Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stages = smem;
@@ -376,6 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5, lane = tid & 31;
     const int TT = p.tile_tokens;
     const int H = p.g.H;
+    const int c0 = blockIdx.x * p.chunk_tokens;  // this CTA's chunk of tokens
+    const int len = min(p.chunk_tokens, p.a.num_tokens - c0);
+    const int ntiles = len > 0 ? (len + TT - 1) / TT : 0;
     if (tid == 0) {
         for (int e = 0; e < kStages; ++e) {
             mbar_init(&full[e], 1);
@@ -396,12 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t pol = policy_evict_first();
         constexpr int kPerLane = (kMaxTileTokens + 31) / 32;
         int sq[kPerLane], po[kPerLane];
-        auto load_ids = [&](int tile, int (&a)[kPerLane], int (&b)[kPerLane]) {
+        auto load_ids = [&](int j, int (&a)[kPerLane], int (&b)[kPerLane]) {
+            const Tile tl = tile_of(c0, len, TT, j);
 #pragma unroll
             for (int r = 0; r < kPerLane; ++r) {
                 const int tt = lane + 32 * r;
-                const int t = tile * TT + tt;
-                const bool in = tile < p.num_tiles && tt < TT && t < p.a.num_tokens;
+                const int t = tl.first + tt;
+                const bool in = tt < tl.count;
                 a[r] = in ? __ldg(p.a.tok_seq + t) : -1;
                 b[r] = in ? __ldg(p.a.tok_pos + t) : -1;
             }
@@ -415,11 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     flag_error(p.err, kErrTimeout);
             }
         };
-        load_ids(blockIdx.x, sq, po);
-        int seqno = 0, n = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++n) {
+        load_ids(0, sq, po);
+        int seqno = 0;
+        for (int n = 0; n < ntiles; ++n) {
+            const Tile tl = tile_of(c0, len, TT, n);
+            // a short tile within the short maps' box takes them: its copy is its own rows
+            const bool short_box = tl.count <= p.short_tokens;
             int nsq[kPerLane], npo[kPerLane];
-            load_ids(tile + gridDim.x, nsq, npo);
+            load_ids(n + 1, nsq, npo);
             int es[2];
             for (int kv = 0; kv < 2; ++kv, ++seqno) {
                 const int e = seqno % kStages;
@@ -438,11 +466,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     return;
                 }
                 if (lane == 0) {
-                    const CUtensorMap* map = kv ? &vmap : &kmap;
+                    const CUtensorMap* map = short_box ? (kv ? &vmap_s : &kmap_s) : (kv ? &vmap : &kmap);
                     uint8_t* dst = stages + e * kStageBytes;
-                    mbar_expect_tx(&full[e], kStageBytes);
-                    tma_load_3d(dst, map, &full[e], 0, 0, tile * kRows, pol);
-                    tma_load_3d(dst + kHalfBytes, map, &full[e], 0, 1, tile * kRows, pol);
+                    // a box counts its full size in bytes, rows past the input's end included
+                    mbar_expect_tx(&full[e], short_box ? uint32_t(p.short_tokens * H) * 256u : uint32_t(kStageBytes));
+                    tma_load_3d(dst, map, &full[e], 0, 0, tl.first * H, pol);
+                    tma_load_3d(dst + kHalfBytes, map, &full[e], 0, 1, tl.first * H, pol);
                 }
             }
             // the meta slot of tile n was last read for tile n - 2, whose stages the waits above freed
@@ -452,9 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int r = 0; r < kPerLane; ++r) {
                 const int tt = lane + 32 * r;
                 if (tt < TT) {
-                    const int t = tile * TT + tt;
                     int2 m = make_int2(-1, 0);
-                    if (t < p.a.num_tokens) {
+                    if (tt < tl.count) {
                         const int sid = sq[r], pos = po[r];
                         bool ok = sid >= 0 && sid < p.a.num_seqs && pos >= 0 && pos / p.g.page_size < p.a.pt_stride &&
                                   (!ROPE || pos < p.g.rope_positions);
@@ -486,8 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------- consumer warps: thread tid owns row tid of each stage ----------------
     const int tt = tid / H, h = tid % H;
-    int seqno = 0, n = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++n) {
+    int seqno = 0;
+    for (int n = 0; n < ntiles; ++n) {
+        const Tile tl = tile_of(c0, len, TT, n);
         int2 m = make_int2(-1, 0);
 #pragma unroll 1
         for (int kv = 0; kv < 2; ++kv, ++seqno) {
@@ -503,8 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float* cs = (ROPE && kv == 0 && m.x >= 0)
                                   ? p.g.rope + int64_t(mpos[(n & 1) * kMaxTileTokens + tt]) * kHeadDim
                                   : nullptr;
-            const int t = tile * TT + tt;
-            if (t < p.a.num_tokens && m.x >= 0) {
+            if (tt < tl.count && m.x >= 0) {
                 const uint8_t* stage = stages + e * kStageBytes;
                 const int64_t row = (int64_t(m.x) * H + h) * p.g.page_size + m.y;
                 if (MODE == 0) {
@@ -543,65 +571,80 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [T*H rows, 2 halves, 64 bf16] view of a [T, H, 128] bf16 input; box = one
-// 128-byte half of kRows consecutive rows, 128-byte swizzle.
-bool make_row_map(CUtensorMap* map, const void* base, int64_t rows) {
+// 128-byte half of box_rows consecutive rows, 128-byte swizzle.
+bool make_row_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {64, 2, cuuint64_t(rows)};
     cuuint64_t strides[2] = {128, 256};
-    cuuint32_t box[3] = {64, 1, kRows};
+    cuuint32_t box[3] = {64, 1, cuuint32_t(box_rows)};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+struct Maps {
+    CUtensorMap k, v;    // whole tiles: kRows rows
+    CUtensorMap ks, vs;  // short tiles: short_tokens * H rows
+};
+
 template <int MODE, int BLK, bool ROTV, bool ROPE, int CB>
-cudaError_t launch_r(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
+cudaError_t launch_r(const Maps& m, const Params& p, int grid, cudaStream_t s) {
     constexpr auto kern = append_kernel<MODE, BLK, ROTV, ROPE, CB>;
     const cudaError_t e = ensure_smem_opt_in<kern>(kSmemBytes);
     if (e != cudaSuccess) return e;
-    return launch_overlapped(kern, dim3(grid), dim3(kThreads), kSmemBytes, s, km, vm, p);
+    return launch_overlapped(kern, dim3(grid), dim3(kThreads), kSmemBytes, s, m.k, m.v, m.ks, m.vs, p);
 }
 
 template <int MODE, int BLK, bool ROTV, bool ROPE>
-cudaError_t launch_c(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
-    if (MODE != 0 && p.g.code_bits == 2) return launch_r<MODE, BLK, ROTV, ROPE, 2>(km, vm, p, grid, s);
-    return launch_r<MODE, BLK, ROTV, ROPE, 4>(km, vm, p, grid, s);
+cudaError_t launch_c(const Maps& m, const Params& p, int grid, cudaStream_t s) {
+    if (MODE != 0 && p.g.code_bits == 2) return launch_r<MODE, BLK, ROTV, ROPE, 2>(m, p, grid, s);
+    return launch_r<MODE, BLK, ROTV, ROPE, 4>(m, p, grid, s);
 }
 
 template <int MODE, int BLK, bool ROTV>
-cudaError_t launch_t(const CUtensorMap& km, const CUtensorMap& vm, const Params& p, int grid, cudaStream_t s) {
-    return p.g.rope ? launch_c<MODE, BLK, ROTV, true>(km, vm, p, grid, s)
-                    : launch_c<MODE, BLK, ROTV, false>(km, vm, p, grid, s);
+cudaError_t launch_t(const Maps& m, const Params& p, int grid, cudaStream_t s) {
+    return p.g.rope ? launch_c<MODE, BLK, ROTV, true>(m, p, grid, s) : launch_c<MODE, BLK, ROTV, false>(m, p, grid, s);
 }
 
 }  // namespace
 
 cudaError_t launch_append(const CacheGeom& g, const AppendArgs& a, int* err_word, int num_sms, cudaStream_t s) {
     if (a.num_tokens == 0) return cudaSuccess;
+    if (num_sms < 1) return cudaErrorInvalidValue;
     const int64_t rows = int64_t(a.num_tokens) * g.H;
-    CUtensorMap km, vm;
-    if (!make_row_map(&km, a.k, rows) || !make_row_map(&vm, a.v, rows)) return cudaErrorInvalidValue;
     Params p;
     p.g = g;
     p.a = a;
     p.tile_tokens = kRows / g.H;
-    p.num_tiles = int((rows + kRows - 1) / kRows);
+    // equal chunks of ceil(T / SMs) tokens; grid = the chunks that hold tokens
+    p.chunk_tokens = (a.num_tokens + num_sms - 1) / num_sms;
+    const int grid = (a.num_tokens + p.chunk_tokens - 1) / p.chunk_tokens;
+    p.short_tokens = p.chunk_tokens % p.tile_tokens;
     p.r_b = g.mode == 2 ? float(1.0 / sqrt(double(g.bdr_block))) : 1.0f;
     p.err = err_word;
-    const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-    if (g.mode == 0) return launch_t<0, 128, false>(km, vm, p, grid, s);
-    if (g.mode == 1) return launch_t<1, 128, false>(km, vm, p, grid, s);
+    Maps m;
+    if (!make_row_map(&m.k, a.k, rows, kRows) || !make_row_map(&m.v, a.v, rows, kRows)) return cudaErrorInvalidValue;
+    if (p.short_tokens > 0) {
+        if (!make_row_map(&m.ks, a.k, rows, p.short_tokens * g.H) ||
+            !make_row_map(&m.vs, a.v, rows, p.short_tokens * g.H))
+            return cudaErrorInvalidValue;
+    } else {  // never taken (no tile has count <= 0); passed so that every parameter is a valid map
+        m.ks = m.k;
+        m.vs = m.v;
+    }
+    if (g.mode == 0) return launch_t<0, 128, false>(m, p, grid, s);
+    if (g.mode == 1) return launch_t<1, 128, false>(m, p, grid, s);
     switch (g.bdr_block * 2 + (g.rotate_v ? 1 : 0)) {
-        case 32: return launch_t<2, 16, false>(km, vm, p, grid, s);
-        case 33: return launch_t<2, 16, true>(km, vm, p, grid, s);
-        case 64: return launch_t<2, 32, false>(km, vm, p, grid, s);
-        case 65: return launch_t<2, 32, true>(km, vm, p, grid, s);
-        case 128: return launch_t<2, 64, false>(km, vm, p, grid, s);
-        case 129: return launch_t<2, 64, true>(km, vm, p, grid, s);
-        case 256: return launch_t<2, 128, false>(km, vm, p, grid, s);
-        case 257: return launch_t<2, 128, true>(km, vm, p, grid, s);
+        case 32: return launch_t<2, 16, false>(m, p, grid, s);
+        case 33: return launch_t<2, 16, true>(m, p, grid, s);
+        case 64: return launch_t<2, 32, false>(m, p, grid, s);
+        case 65: return launch_t<2, 32, true>(m, p, grid, s);
+        case 128: return launch_t<2, 64, false>(m, p, grid, s);
+        case 129: return launch_t<2, 64, true>(m, p, grid, s);
+        case 256: return launch_t<2, 128, false>(m, p, grid, s);
+        case 257: return launch_t<2, 128, true>(m, p, grid, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -54,6 +54,46 @@ def test_append_ragged_shapes(H, ps, lengths):
         assert_pools_equal(c)
 
 
+def _chunk_case_tokens(S, TT, whole, short, last):
+    """Token count whose per-CTA chunks are `whole` tiles + `short` tokens on S SMs, the last chunk
+    `last` tokens."""
+    Tc = whole * TT + short
+    N = (S - 1) * Tc + last
+    assert 1 <= last <= Tc and -(-N // S) == Tc
+    return N
+
+
+# (H, whole tiles per chunk, short tokens, last chunk's tokens): the last chunk's remainder above
+# the short box (it takes the whole-tile box) or within it, chunks of one short tile, other H
+CHUNK_CASES = [(8, 1, 1, 21), (8, 2, 19, 42), (8, 0, 5, 5), (2, 1, 30, 10), (32, 3, 2, 6)]
+
+
+@pytest.mark.parametrize("H,whole,short,last", CHUNK_CASES, ids=[f"H{c[0]}_w{c[1]}_s{c[2]}_l{c[3]}" for c in CHUNK_CASES])
+def test_append_chunk_schedule(H, whole, short, last):
+    """Each CTA appends a contiguous chunk of ceil(T / SMs) tokens: a short first tile (its own
+    small TMA box) when the chunk is not whole tiles, then whole tiles of 224 / H tokens."""
+    S = torch.cuda.get_device_properties(0).multi_processor_count
+    N = _chunk_case_tokens(S, 224 // H, whole, short, last)
+    lengths = [N // 3, N // 3, N - 2 * (N // 3)]
+    wl = synth.Workload("t", H, 4 * H if H <= 32 else H, 128, 16, synth.OUTLIERS_X20, "test")
+    for mode, b, rv in ((kvq.KV_INT4_BDR, 128, True), (kvq.KV_BF16, 0, False)):
+        c = make_case(mode, b, rv, lengths, wl, seed=N + H)
+        assert gpu_append(c) == kvq.KV_OK
+        assert oracle_append(c) == 0
+        assert_pools_equal(c)
+
+
+def test_append_fewer_tokens_than_sms():
+    """Fewer tokens than SMs: one token per CTA, each a short tile of H rows."""
+    S = torch.cuda.get_device_properties(0).multi_processor_count
+    wl = synth.Workload("t", 8, 32, 128, 16, synth.OUTLIERS_X20, "test")
+    for mode, b, rv in ((kvq.KV_INT4_BDR, 64, False), (kvq.KV_INT4, 0, False)):
+        c = make_case(mode, b, rv, [S // 2, S // 3], wl, seed=5)
+        assert gpu_append(c) == kvq.KV_OK
+        assert oracle_append(c) == 0
+        assert_pools_equal(c)
+
+
 def test_append_empty_is_noop():
     c = make_case(kvq.KV_INT4_BDR, 128, False, [4], WL0)
     e = torch.empty(0, 8, 128, dtype=torch.bfloat16, device="cuda")
