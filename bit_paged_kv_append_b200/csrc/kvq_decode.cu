@@ -20,8 +20,7 @@
 namespace kvq {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kWarps = kThreads / 32;
+constexpr int kMergeWarps = 4;  // (sequence, query head) rows per merge CTA, one warp each
 using Params = DecodeParams;
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -37,81 +36,108 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ---------------------------------------------------------------- merge --------
 
-// One CTA per (sequence, query head): merge the sequence's splits (statistics
-// fetched once, 128 splits at a time, partial outputs loaded 8 at a time),
-// normalise, rotate back
-// when values were rotated (o H_blk; H_blk is its own inverse), store bf16 (round
-// to nearest even of the fp32 value) or fp32.  An empty sequence gives zeros.
-__global__ void __launch_bounds__(kThreads) merge_kernel(Params p, int rotate_out) {
-    __shared__ float wts[kThreads];
-    __shared__ float red[2][kWarps];
-    __shared__ float buf[kHeadDim];
-    const int row = blockIdx.x;  // s * Hq + j
+// One warp per (sequence, query head) row, lane l owning dims 4l .. 4l + 3: merge the
+// sequence's splits (statistics 32 splits at a time, one per lane, their maximum and
+// weighted sum by shuffles; partial outputs 8 splits at a time as float4), normalise,
+// rotate back when values were rotated (o H_blk; H_blk is its own inverse: butterflies of
+// stride 1 and 2 within a lane, 4 .. 64 across lanes), store bf16 (round to nearest even
+// of the fp32 value) or fp32.  An empty sequence gives zeros.  No block barrier: a warp
+// finishes its row alone.
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(Params p, int rotate_out) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Hq = p.g.Hq;
-    const int s = row / Hq, j = row % Hq;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int row = blockIdx.x * kMergeWarps + warp;  // s * Hq + j
     grid_dep_wait();  // the split kernel's partials
     grid_dep_launch();
+    if (row >= p.a.batch * Hq) return;  // whole warps
+    const int s = row / Hq, j = row % Hq;
     const int n = (decode_len(p, s) + p.item_tokens - 1) / p.item_tokens;
-    const int64_t stride = int64_t(Hq) * kHeadDim;  // next split, same query head
-    float acc = 0.0f, l = 0.0f, M = -INFINITY;
-    // splits in tiles of 128: thread t fetches the statistics of split k0 + t, the tile's
-    // weights go through shared memory, every thread then sums its dimension over the tile
-    for (int k0 = 0; k0 < n; k0 += kThreads) {
-        const int cnt = min(kThreads, n - k0);
-        const float2 ml = tid < cnt ? p.ws_ml[partial_row(p, s, k0 + tid, j)] : make_float2(-INFINITY, 0.0f);
-        float tm = warp_max(ml.x);
-        if (lane == 0) red[0][warp] = tm;
-        __syncthreads();
-        tm = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
-        const float Mn = fmaxf(M, tm);
-        const float f = (ml.x == -INFINITY) ? 0.0f : fast_exp2(ml.x - Mn);
-        wts[tid] = f;
-        const float lt = warp_sum(f * ml.y);
-        if (lane == 0) red[1][warp] = lt;
-        __syncthreads();
+    const int64_t stride4 = int64_t(Hq) * (kHeadDim / 4);  // next split, same query head, in float4
+    float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float l = 0.0f, M = -INFINITY;
+    for (int k0 = 0; k0 < n; k0 += 32) {
+        const int cnt = min(32, n - k0);
+        const float2 ml = lane < cnt ? p.ws_ml[partial_row(p, s, k0 + lane, j)] : make_float2(-INFINITY, 0.0f);
+        const float Mn = fmaxf(M, warp_max(ml.x));
+        const float f = (ml.x == -INFINITY) ? 0.0f : fast_exp2(ml.x - Mn);  // this lane's split weight
         const float rescale = (M == -INFINITY) ? 0.0f : fast_exp2(M - Mn);
-        l = l * rescale + (red[1][0] + red[1][1] + red[1][2] + red[1][3]);
-        acc *= rescale;
+        l = l * rescale + warp_sum(f * ml.y);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c] *= rescale;
         M = Mn;
-        const float* src = p.ws_o + partial_row(p, s, k0, j) * kHeadDim + tid;
+        const float4* src = reinterpret_cast<const float4*>(p.ws_o + partial_row(p, s, k0, j) * kHeadDim) + lane;
         int t = 0;
         for (; t + 8 <= cnt; t += 8) {
-            float o[8];
+            float4 o[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) o[u] = src[(t + u) * stride];
+            for (int u = 0; u < 8; ++u) o[u] = src[(t + u) * stride4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) acc += wts[t + u] * o[u];
+            for (int u = 0; u < 8; ++u) {
+                const float w = __shfl_sync(0xffffffffu, f, t + u);
+                v[0] += w * o[u].x;
+                v[1] += w * o[u].y;
+                v[2] += w * o[u].z;
+                v[3] += w * o[u].w;
+            }
         }
-        for (; t < cnt; ++t) acc += wts[t] * src[t * stride];
-        __syncthreads();
+        for (; t < cnt; ++t) {
+            const float4 o = src[t * stride4];
+            const float w = __shfl_sync(0xffffffffu, f, t);
+            v[0] += w * o.x;
+            v[1] += w * o.y;
+            v[2] += w * o.z;
+            v[3] += w * o.w;
+        }
     }
-    float res = l > 0.0f ? acc / l : 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) v[c] = l > 0.0f ? v[c] / l : 0.0f;
     if (rotate_out) {
-        buf[tid] = res;
-        __syncthreads();
-        for (int hs = 1; hs < p.g.bdr_block; hs <<= 1) {
-            const float mine = buf[tid], other = buf[tid ^ hs];
-            const float nv = (tid & hs) ? other - mine : mine + other;
-            __syncthreads();
-            buf[tid] = nv;
-            __syncthreads();
+        const int b = p.g.bdr_block;  // 16 .. 128
+        // element 4 lane + c; at stride hs the lower element of each pair takes a + d, the
+        // upper a - d
+#pragma unroll
+        for (int hs = 1; hs < 4; hs <<= 1) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if ((c & hs) == 0) {
+                    const float a = v[c], d = v[c + hs];
+                    v[c] = a + d;
+                    v[c + hs] = a - d;
+                }
+            }
         }
-        res = buf[tid] * rsqrtf(float(p.g.bdr_block));
+        for (int hs = 4; hs < b; hs <<= 1) {
+            const int ls = hs >> 2;  // partner lane distance
+            const bool upper = (lane & ls) != 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float other = __shfl_xor_sync(0xffffffffu, v[c], ls);
+                v[c] = upper ? other - v[c] : v[c] + other;
+            }
+        }
+        const float r = rsqrtf(float(b));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c] *= r;
     }
-    const int64_t o = int64_t(row) * kHeadDim + tid;
-    if (p.a.out_fp32)
-        static_cast<float*>(p.a.out)[o] = res;
-    else
-        static_cast<__nv_bfloat16*>(p.a.out)[o] = __float2bfloat16_rn(res);
+    const int64_t o = int64_t(row) * kHeadDim + 4 * lane;  // out is 16-byte aligned (checked by the API)
+    if (p.a.out_fp32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(p.a.out) + o) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&lo);
+        w.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.a.out) + o) = w;
+    }
 }
 
 template <int G>
 cudaError_t launch_group(const Params& p, cudaStream_t st) {
     const cudaError_t e = p.g.mode == 0 ? launch_decode_bf16(p, st) : launch_decode_mma(p, st);
     if (e != cudaSuccess) return e;
-    return launch_overlapped(merge_kernel, dim3(p.a.batch * p.g.Hq), dim3(kThreads), 0, st, p,
-                             int(p.g.mode == 2 && p.g.rotate_v));
+    const int rows = p.a.batch * p.g.Hq;
+    return launch_overlapped(merge_kernel, dim3((rows + kMergeWarps - 1) / kMergeWarps), dim3(kMergeWarps * 32), 0,
+                             st, p, int(p.g.mode == 2 && p.g.rotate_v));
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

@@ -7,7 +7,7 @@
 //          of sequence s -> unnormalised partial output + softmax statistics
 //          (kvq_decode_mma.cu for INT4 pages, kvq_decode.cu for BF16 pages);
 //          CTAs past the end of their sequence exit at once.
-//   merge  one CTA per (sequence, query head): log-sum-exp merge of its splits,
+//   merge  one warp per (sequence, query head): log-sum-exp merge of its splits,
 //          output rotation, bf16/fp32 store (kvq_decode.cu).
 #pragma once
 
