@@ -38,26 +38,35 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // One warp per (sequence, query head) row, lane l owning dims 4l .. 4l + 3: merge the
 // sequence's splits (statistics 32 splits at a time, one per lane, their maximum and
-// weighted sum by shuffles; partial outputs 8 splits at a time as float4), normalise,
-// rotate back when values were rotated (o H_blk; H_blk is its own inverse: butterflies of
-// stride 1 and 2 within a lane, 4 .. 64 across lanes), store bf16 (round to nearest even
-// of the fp32 value) or fp32.  An empty sequence gives zeros.  No block barrier: a warp
-// finishes its row alone.
-__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(Params p, int rotate_out) {
+// weighted sum by shuffles, the next pass's statistics fetched before this pass's rows;
+// partial outputs 8 splits at a time as float4), normalise, rotate back when values were
+// rotated (o H_blk; H_blk is its own inverse: butterflies of stride 1 and 2 within a
+// lane, 4 .. 64 across lanes), store bf16 (round to nearest even of the fp32 value) or
+// fp32.  An empty sequence gives zeros.  With share_rows (few rows of many splits) the
+// CTA's warps share one row, warp w taking passes w, w + 4, ..., and warp 0 combines
+// their (max, sum, vector) through shared memory; otherwise each warp finishes its row
+// alone, with no block barrier.
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(Params p, int rotate_out, int share_rows) {
+    __shared__ float4 part_v[kMergeWarps][32];
+    __shared__ float2 part_ml[kMergeWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Hq = p.g.Hq;
-    const int row = blockIdx.x * kMergeWarps + warp;  // s * Hq + j
+    const int row = share_rows ? blockIdx.x : blockIdx.x * kMergeWarps + warp;  // s * Hq + j
+    const int k_first = share_rows ? 32 * warp : 0;
+    const int k_step = share_rows ? 32 * kMergeWarps : 32;
     grid_dep_wait();  // the split kernel's partials
     grid_dep_launch();
-    if (row >= p.a.batch * Hq) return;  // whole warps
+    if (row >= p.a.batch * Hq) return;  // whole warps (with share_rows, the whole CTA)
     const int s = row / Hq, j = row % Hq;
     const int n = (decode_len(p, s) + p.item_tokens - 1) / p.item_tokens;
     const int64_t stride4 = int64_t(Hq) * (kHeadDim / 4);  // next split, same query head, in float4
     float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     float l = 0.0f, M = -INFINITY;
-    for (int k0 = 0; k0 < n; k0 += 32) {
+    float2 ml = k_first + lane < n ? p.ws_ml[partial_row(p, s, k_first + lane, j)] : make_float2(-INFINITY, 0.0f);
+    for (int k0 = k_first; k0 < n; k0 += k_step) {
         const int cnt = min(32, n - k0);
-        const float2 ml = lane < cnt ? p.ws_ml[partial_row(p, s, k0 + lane, j)] : make_float2(-INFINITY, 0.0f);
+        const int kn = k0 + k_step + lane;
+        const float2 ml_next = kn < n ? p.ws_ml[partial_row(p, s, kn, j)] : make_float2(-INFINITY, 0.0f);
         const float Mn = fmaxf(M, warp_max(ml.x));
         const float f = (ml.x == -INFINITY) ? 0.0f : fast_exp2(ml.x - Mn);  // this lane's split weight
         const float rescale = (M == -INFINITY) ? 0.0f : fast_exp2(M - Mn);
@@ -65,6 +74,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(Params p, int r
 #pragma unroll
         for (int c = 0; c < 4; ++c) v[c] *= rescale;
         M = Mn;
+        ml = ml_next;
         const float4* src = reinterpret_cast<const float4*>(p.ws_o + partial_row(p, s, k0, j) * kHeadDim) + lane;
         int t = 0;
         for (; t + 8 <= cnt; t += 8) {
@@ -87,6 +97,29 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(Params p, int r
             v[1] += w * o.y;
             v[2] += w * o.z;
             v[3] += w * o.w;
+        }
+    }
+    if (share_rows) {
+        part_v[warp][lane] = make_float4(v[0], v[1], v[2], v[3]);
+        if (lane == 0) part_ml[warp] = make_float2(M, l);
+        __syncthreads();
+        if (warp != 0) return;
+        float Mt = part_ml[0].x;
+#pragma unroll
+        for (int w = 1; w < kMergeWarps; ++w) Mt = fmaxf(Mt, part_ml[w].x);
+        l = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c] = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) {
+            const float2 wm = part_ml[w];
+            const float f = (wm.x == -INFINITY) ? 0.0f : fast_exp2(wm.x - Mt);
+            const float4 pv = part_v[w][lane];
+            l += f * wm.y;
+            v[0] += f * pv.x;
+            v[1] += f * pv.y;
+            v[2] += f * pv.z;
+            v[3] += f * pv.w;
         }
     }
 #pragma unroll
@@ -132,12 +165,16 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(Params p, int r
 }
 
 template <int G>
-cudaError_t launch_group(const Params& p, cudaStream_t st) {
+cudaError_t launch_group(const Params& p, int num_sms, cudaStream_t st) {
     const cudaError_t e = p.g.mode == 0 ? launch_decode_bf16(p, st) : launch_decode_mma(p, st);
     if (e != cudaSuccess) return e;
+    // few rows of more than one pass of splits (long sequences, small batches): the CTA's
+    // warps share a row
     const int rows = p.a.batch * p.g.Hq;
-    return launch_overlapped(merge_kernel, dim3((rows + kMergeWarps - 1) / kMergeWarps), dim3(kMergeWarps * 32), 0,
-                             st, p, int(p.g.mode == 2 && p.g.rotate_v));
+    const int share = p.max_splits > 32 && rows <= 4 * (num_sms > 0 ? num_sms : 148);
+    const int grid = share ? rows : (rows + kMergeWarps - 1) / kMergeWarps;
+    return launch_overlapped(merge_kernel, dim3(grid), dim3(kMergeWarps * 32), 0, st, p,
+                             int(p.g.mode == 2 && p.g.rotate_v), share);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -187,10 +224,10 @@ cudaError_t launch_decode(const CacheGeom& g, const DecodeArgs& a, const DecodeP
     p.ws_ml = reinterpret_cast<float2*>(ws + align256(rows * kHeadDim * sizeof(float)));
     p.err = err_word;
     switch (g.Hq / g.H) {
-        case 1: return launch_group<1>(p, s);
-        case 2: return launch_group<2>(p, s);
-        case 4: return launch_group<4>(p, s);
-        case 8: return launch_group<8>(p, s);
+        case 1: return launch_group<1>(p, plan.num_sms, s);
+        case 2: return launch_group<2>(p, plan.num_sms, s);
+        case 4: return launch_group<4>(p, plan.num_sms, s);
+        case 8: return launch_group<8>(p, plan.num_sms, s);
         default: return cudaErrorInvalidValue;
     }
 }

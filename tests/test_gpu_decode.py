@@ -73,6 +73,30 @@ def test_decode_long_sequence_many_splits(mode, b):
     _run(c, lengths)
 
 
+def test_decode_long_rows_shared_by_merge_warps():
+    """More than 32 splits per row and few rows: the merge CTA's four warps share each row (the
+    40k-token row has three passes of 32 splits, so one warp holds none) and warp 0 combines
+    them; values rotated, so the merged output is turned back; an empty and a short sequence in
+    the same batch."""
+    wl = synth.Workload("t", 8, 32, 128, 64, synth.OUTLIERS_1PCT, "test")
+    c = make_case(kvq.KV_INT4_BDR, 64, True, [40_000, 1, 3000], wl, seed=4)
+    assert gpu_append(c) == kvq.KV_OK
+    oracle_append(c)
+    assert_pools_equal(c)
+    lengths = [40_000, 0, 3000]
+    q = synth.make_q(3, 32, 128, seed=9)
+    ref, skipped = oracle_decode(c, q, lengths)
+    assert skipped == 0
+    out32, st = gpu_decode(c, q, lengths, out_fp32=True)
+    assert st == kvq.KV_OK
+    o = out32.cpu().numpy()
+    assert not o[1].any()
+    assert attn_rel_err(o, ref) <= ATTN_RTOL
+    out16, st = gpu_decode(c, q, lengths, out_fp32=False)
+    assert st == kvq.KV_OK
+    assert torch.equal(out16, out32.to(torch.bfloat16))
+
+
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_decode_bf16_group_sizes_nan_filled_pool(G):
     """BF16 pages, every group size.  The pools hold NaN bits before the append, so the slots
