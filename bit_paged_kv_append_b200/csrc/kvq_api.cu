@@ -96,6 +96,7 @@ kv_status kv_append_quant(kv_cache* c, const void* k, const void* v, int num_tok
         !aligned(page_table, 4))
         return KV_ERR_INVALID;
     if (pt_stride < 1 || num_seqs < 1) return KV_ERR_INVALID;
+    if (int64_t(num_tokens) * c->g.H > INT32_MAX) return KV_ERR_INVALID;  // rows index the TMA box as int32
     kvq::AppendArgs a{k, v, num_tokens, tok_seq, tok_pos, page_table, pt_stride, num_seqs};
     kvq::DeviceGuard dg(c->device);
     if (!dg.ok()) return KV_ERR_CUDA;

@@ -131,8 +131,9 @@ kv_status kv_create_paged(const kv_desc* desc, kv_cache** out);
  *  tok_pos     device int32 [num_tokens]: its position within that sequence
  *  page_table  device int32 [num_seqs, pt_stride]
  * Two tokens must not target the same slot in one call.  num_tokens == 0 is a
- * no-op.  Out-of-range sequence ids, positions or page ids are skipped and
- * flagged (KV_ERR_OOB via kv_get_error). */
+ * no-op; num_tokens * num_kv_heads above INT32_MAX rows is KV_ERR_INVALID.
+ * Out-of-range sequence ids, positions or page ids are skipped and flagged
+ * (KV_ERR_OOB via kv_get_error). */
 kv_status kv_append_quant(kv_cache* cache, const void* k, const void* v, int num_tokens,
                           const int32_t* tok_seq, const int32_t* tok_pos, const int32_t* page_table,
                           int pt_stride, int num_seqs, void* stream);
